@@ -1,0 +1,384 @@
+"""Benchmark: routed tokens/s of the router step (router GEMM + sigmoid + biased
+Top-K + gates + load histogram + SMEBU update) on the tie workload
+(T=1,048,576 tokens, d=4096, N_r=256, K=4, hidden on a 1/8 grid, 8 experts
+starting at bias -1.0), GEMM mode, bf16 inputs with fp32 accumulation.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Each rank routes its own batch of T
+tokens (weak scaling); the per-expert loads are summed across ranks with one
+NCCL all-reduce before the SMEBU step, so every rank applies the same update.
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle on the
+host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "ties"
+METRIC = "routed tokens/s (router+top-K+hist+SMEBU) at N_r=256,K=4; % of roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-full-step", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+ROUTER_SOURCES = ["expert_bias_load_b200/csrc/router_gemm.cu", "expert_bias_load_b200/csrc/ptx.cuh",
+                  "expert_bias_load_b200/csrc/topk.cuh"]
+
+
+def profiled_traffic(workload_key):
+    """DRAM bytes per launch of the router kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "router_gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("source_hash") != kernel_source_hash(ROUTER_SOURCES):
+        return None
+    entry = j.get("per_launch", {}).get(workload_key)
+    return None if entry is None else float(entry["dram_bytes_full_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle leg
+
+def oracle_sample(cfg, seconds, seed=0):
+    """Time the CPU oracle (router in fp64 + SMEBU) on a bounded sample of the
+    workload's rows; returns (tokens_per_s, rows, threads, seconds)."""
+    import numpy as np
+    import oracle
+    import synth
+    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
+    oracle.build()
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d)
+    bias = synth.dead_start_bias(Nr).numpy()
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+    def run(rows):
+        h = synth.hidden_normal(rows, d, seed=seed + rows, quant8=True)
+        b = bias.copy()
+        m = np.zeros(Nr, np.float32)
+        t0 = time.perf_counter()
+        r = oracle.router_gemm(h, W, b, K)
+        oracle.smebu(r.counts, b, m)
+        return time.perf_counter() - t0
+
+    rows = 64
+    t = run(rows)
+    rows = int(max(64, min(T, rows * seconds / max(t, 1e-3))))
+    t = run(rows)
+    return rows / t, rows, threads, t
+
+
+# ------------------------------------------------------------------- GPU leg
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    import synth
+    cfg = synth.WORKLOADS[WORKLOAD]
+    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
+    config = {"workload": "tie workload: T=%d tokens/GPU, d=%d, N_r=%d, K=%d, hidden on a 1/8 grid, "
+                          "8 experts at bias -1.0, GEMM mode" % (T, d, Nr, K),
+              "tokens_per_gpu": T, "d": d, "N_r": Nr, "K": K, "smebu": [5e-4, 0.5, 2.0],
+              "l2": "inputs larger than L2 (hidden %.1f GB per GPU)" % (T * d * 2 / 1e9),
+              "parallelism": "dp%d (per-expert loads all-reduced)" % world}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        rows = threads = None
+        for s in range(args.warmup + args.steps):
+            v, rows, threads, secs = oracle_sample(cfg, max(1.0, args.cpu_seconds / 4), seed=s)
+            if s >= args.warmup:
+                vals.append(v)
+        v = statistics.median(vals)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": rows / v * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                 "sample": "%d rows of the tie workload per step (fp64 router + SMEBU)" % rows},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import expert_bias_load_b200 as ebl
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ebl.lib()
+
+    # inputs resident in HBM: a fresh seeded batch per rank
+    h = synth.hidden_normal(T, d, seed=synth.step_seed(WORKLOAD, 0) + 1000 * rank, device=dev, quant8=True)
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    bias = synth.dead_start_bias(Nr, device=dev)
+    mom = torch.zeros(Nr, device=dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    gates = torch.empty(T, K, dtype=torch.float32, device=dev)
+    maxvio = torch.zeros(1, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev0=None, ev1=None):
+        if ev0 is not None:
+            ev0.record(stream)
+        ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=gates, status=status, stream=stream)
+        if ev1 is not None:
+            ev1.record(stream)
+        if world > 1:
+            dist.all_reduce(counts)
+        ebl.smebu_step(counts, bias, mom, reset_counts=True, maxvio=maxvio, status=status, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    maxvio_first = float(maxvio.item())
+
+    evr = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(*evr[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = e0.elapsed_time(e1)
+    router_ms = statistics.mean(a.elapsed_time(b) for a, b in evr)
+    if world > 1:
+        t = torch.tensor([total_ms, router_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, router_ms = float(t[0]), float(t[1])
+    st = int(status.item())
+    ms_step = total_ms / args.steps
+    value = T * world / (ms_step / 1e3)
+
+    peaks = measured_peaks()
+    flops = 2.0 * T * d * Nr
+    alg_bytes = 2.0 * T * d + 8.0 * T * K + 2.0 * Nr * d + 8.0 * Nr
+    achieved = flops / (router_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic("ties_full"),
+                "kernel": "router_gemm_kernel<4>", "kernel_ms": router_ms,
+                "peak_source": "%s burst bf16 (MEASURED_PEAKS.json)" % peaks["source"],
+                "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                "hbm_view": {"alg_bytes": alg_bytes, "achieved_gbs": alg_bytes / (router_ms / 1e3) / 1e9,
+                             "peak_gbs": peaks["hbm_gbs"],
+                             "frac": alg_bytes / (router_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+                "roofline_time_ms": max(flops / peaks["bf16_tflops"] / 1e12, alg_bytes / peaks["hbm_gbs"] / 1e9) * 1e3}
+    roofline["frac_of_roofline_step"] = roofline["roofline_time_ms"] / ms_step
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        h_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+        h_host.copy_(h)
+        idx_host = torch.empty((T, K), dtype=torch.int32, pin_memory=True)
+        gates_host = torch.empty((T, K), dtype=torch.float32, pin_memory=True)
+        state_host = torch.empty((2 * Nr + 1,), dtype=torch.float32, pin_memory=True)
+        state_dev = torch.empty((2 * Nr + 1,), dtype=torch.float32, device=dev)
+
+        def e2e_step():
+            h.copy_(h_host, non_blocking=True)
+            step()
+            state_dev[:Nr].copy_(bias)
+            state_dev[Nr:2 * Nr].copy_(mom)
+            state_dev[2 * Nr:].copy_(maxvio)
+            idx_host.copy_(idx, non_blocking=True)
+            gates_host.copy_(gates, non_blocking=True)
+            state_host.copy_(state_dev, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": T * world / (e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+               "d2h_bytes_per_step": T * K * 8 + (2 * Nr + 1) * 4, "ms_per_step": e_ms}
+        del h_host
+
+    # ---- the rest of the hot path: dispatch, identity expert, combine (same workload)
+    full = None
+    if not args.no_full_step:
+        tiles = torch.empty(((T + 127) // 128, Nr), dtype=torch.int32, device=dev)
+        offsets = torch.empty(Nr + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * K, dtype=torch.int32, device=dev)
+        dest = torch.empty(T * K, dtype=torch.int32, device=dev)
+        X = torch.empty((T * K, d), dtype=torch.bfloat16, device=dev)
+        out = torch.empty((T, d), dtype=torch.float32, device=dev)
+        ws = torch.empty(ebl.dispatch_workspace_bytes(T, Nr), dtype=torch.uint8, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+        def fstep(rec):
+            if rec:
+                ev[0].record(stream)
+            ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=gates, tile_counts=tiles,
+                               status=status, stream=stream)
+            if world > 1:
+                dist.all_reduce(counts)
+            ebl.smebu_step(counts, bias, mom, reset_counts=True, maxvio=maxvio, status=status, stream=stream)
+            if rec:
+                ev[1].record(stream)
+            ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles, offsets=offsets, perm=perm, dest=dest, dispatched=X,
+                             workspace=ws, status=status, stream=stream)
+            if rec:
+                ev[2].record(stream)
+            ebl.moe_combine(X, gates, dest, out=out, status=status, stream=stream)
+            if rec:
+                ev[3].record(stream)
+
+        for _ in range(2):
+            fstep(False)
+        torch.cuda.synchronize()
+        reps = max(3, min(10, args.steps // 50))
+        tr = td = tc = 0.0
+        for _ in range(reps):
+            fstep(True)
+            torch.cuda.synchronize()
+            tr += ev[0].elapsed_time(ev[1])
+            td += ev[1].elapsed_time(ev[2])
+            tc += ev[2].elapsed_time(ev[3])
+        tr, td, tc = tr / reps, td / reps, tc / reps
+        disp_bytes = T * d * 2 + T * K * d * 2
+        comb_bytes = T * K * d * 2 + T * d * 4
+        full = {"metric": "tokens/s through router+SMEBU+dispatch+identity expert+combine",
+                "value": T * world / ((tr + td + tc) / 1e3), "ms_per_step": tr + td + tc,
+                "router_smebu_ms": tr, "dispatch_ms": td, "combine_ms": tc,
+                "dispatch_gbs": disp_bytes / (td / 1e3) / 1e9, "combine_gbs": comb_bytes / (tc / 1e3) / 1e9,
+                "dispatch_frac_hbm": disp_bytes / (td / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "combine_frac_hbm": comb_bytes / (tc / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        del X, out
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, rows, threads, secs = oracle_sample(cfg, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": "%d rows of the tie workload (fp64 router GEMM + top-K + gates + counts, then SMEBU), "
+                         "%.1f s" % (rows, secs)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+            "clocks": clk, "status": st, "maxvio_after_warmup": maxvio_first, "full_step": full}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

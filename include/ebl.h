@@ -1,0 +1,228 @@
+/*
+ * ebl.h -- C ABI of libebl.so: the MoE router step with aux-loss-free
+ * expert-bias balancing (SMEBU), hand-written CUDA for sm_100a (B200).
+ *
+ * The method (page titles, sections and equations):
+ *   "Arcee Trinity Large Technical Report", section 2.3 "Mixture-of-Experts":
+ *     sigmoid routing with normalized scores; Top-K on routing score plus
+ *     expert bias; gates from the routing scores without the bias; SMEBU
+ *     with lambda = 5e-4, beta = 0.5, kappa = 2; the sign update of the
+ *     smaller models; a linear unclamped update as an ablation.
+ *   "SMEBU Load Balancing" (study note), "How it works": eq. (17) bias only
+ *     inside Top-K; eqs. (20)-(22) sign update with re-centred bias;
+ *     eqs. (23)-(28) normalised violation, tanh clamp, scaled and re-centred
+ *     step, momentum, bias add.
+ *   "Arcee Halts 400B Blackwell Model Collapse With Dynamic Router Biases",
+ *     "The MaxVio Metric and the Day-4 Crisis": MaxVio, the ratio of the most-
+ *     to the least-routed expert's load.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers marked "device" are CUDA device pointers (or managed memory) on
+ *     the current device.  The caller owns every buffer; the library keeps no
+ *     pointer after a call returns and allocates no device memory.
+ *   - bf16 data is passed as uint16_t bit patterns (IEEE binary32 upper half).
+ *   - All arrays are dense row-major, innermost index last.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and never synchronises.  Host-side argument checks run before anything
+ *     is launched; a call that returns an error launched nothing, except
+ *     EBL_ECUDA, which reports a launch failure.
+ *   - Return value: EBL_OK (0) or a negative error code (ebl_strerror()).
+ *   - Errors only visible on the device (an expert id out of range, a sum of
+ *     loads of zero, a pipeline wait that ran out) are OR-ed into the optional
+ *     device word `status` as EBL_ST_* bits; kernels never trap.  With
+ *     status == NULL they go to a library-owned device word that
+ *     ebl_read_internal_status() reads.
+ */
+#ifndef EBL_H
+#define EBL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *ebl_stream_t;
+
+/* Return codes. */
+#define EBL_OK 0
+#define EBL_EINVAL (-1)       /* null pointer, bad shape or size, misaligned pointer */
+#define EBL_EUNSUPPORTED (-2) /* valid request this build does not implement (e.g. N_r % 32 != 0 in GEMM mode) */
+#define EBL_ECUDA (-3)        /* a CUDA runtime/driver call failed; the CUDA error is cleared */
+#define EBL_EDATA (-4)        /* reserved for data errors reported synchronously */
+
+/* Bits of the device status word. */
+#define EBL_ST_BAD_EXPERT 1   /* an expert id outside [0, N_r) was seen; that pair was skipped */
+#define EBL_ST_BAD_DEST 2     /* a dest index outside [0, T*K) was seen; that slot was skipped */
+#define EBL_ST_EMPTY_LOAD 4   /* sum of loads was 0: bias/momentum left untouched */
+#define EBL_ST_TIMEOUT 8      /* a pipeline wait inside the router kernel ran out; outputs invalid */
+
+#define EBL_MAX_EXPERTS 256   /* N_r limit of every entry point */
+#define EBL_MAX_TOPK 8        /* K limit */
+
+/* Human-readable text for a return code. Never NULL. */
+const char *ebl_strerror(int code);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ebl_version(void);
+
+/* Tokens per router tile: the row count of one tile_counts row (128). */
+int ebl_tile_tokens(void);
+
+/*
+ * router_forward -- one router pass in GEMM mode.
+ * Passage: "Arcee Trinity Large Technical Report" 2.3 (sigmoid routing with
+ * normalized scores; Top-K on score plus bias; gates without the bias) and
+ * "SMEBU Load Balancing" eq. (17).
+ *
+ * For every token t < T:
+ *   x_{t,i}  = sum_k hidden[t,k] * W_router[i,k]     bf16 x bf16, fp32 accumulate (tensor cores)
+ *   s_{t,i}  = 1 / (1 + exp(-x_{t,i}))               fp32
+ *   key      = s_{t,i} + bias[i]                      fp32, bias used only here
+ *   topk_idx[t, 0..K-1] = the K experts of largest key; equal keys go to the
+ *                         lower expert index; slots sorted by (key desc, index asc)
+ *   gates[t,k] = s_{t,idx_k} / sum_k' s_{t,idx_k'}   (bias-free, sums to 1)
+ *   counts[i] += #{(t,k) : topk_idx[t,k] == i}        ACCUMULATED: the caller zeroes
+ *                                                     counts once per optimizer step
+ *   tile_counts[j, i] = the same count over tokens [128 j, 128 j + 128)  (overwritten)
+ *
+ * hidden       device, bf16 [T, d]; 16-byte aligned.
+ * W_router     device, bf16 [N_r, d] (expert-major, i.e. K-major for the MMA); 16-byte aligned.
+ * bias         device, fp32 [N_r].
+ * T            tokens, 0 <= T <= 2^31 - 2^8.  T == 0 is a no-op.
+ * d            hidden size, d % 64 == 0, 64 <= d <= 2^20.
+ * N_r          routed experts, N_r % 32 == 0, 32 <= N_r <= 256 (else EBL_EUNSUPPORTED).
+ * K            experts per token, 1 <= K <= min(8, N_r).
+ * topk_idx     device, int32 [T, K], written.
+ * gates        device, fp32 [T, K], written.
+ * counts       device, int32 [N_r], accumulated with one atomic per expert per CTA.
+ * tile_counts  device, int32 [ceil(T/128), N_r], written; or NULL to skip.
+ * status       device int32 or NULL; EBL_ST_TIMEOUT if the pipeline stalled.
+ * Inputs are assumed finite.  Deterministic: the outputs do not depend on
+ * scheduling (integer histogram, per-row arithmetic in a fixed order).
+ */
+int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float *bias,
+                   int T, int d, int N_r, int K,
+                   int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                   int32_t *status, ebl_stream_t stream);
+
+/*
+ * router_forward_logits -- the same selection, gates and counts from
+ * precomputed fp32 logits.  This is the bit-exact mode: each value that
+ * decides a selection has one defined rounding,
+ *   s   = (float)(1 / (1 + exp(-(double)x)))        fp64 evaluation, rounded once
+ *   key = s + bias[i]                                one fp32 add, round to nearest
+ *   g_k = (float)((double)s_k / sum_k' (double)s_k')  fp64, slot order, rounded once
+ * so indices, counts and tile_counts match any implementation of these
+ * formulas exactly (up to a last-ulp difference between two fp64 exp
+ * implementations, about one value in 2^28).
+ *
+ * logits  device, fp32 [T, N_r].
+ * N_r     1 <= N_r <= 256 (any value).  K: 1 <= K <= min(8, N_r).
+ * Other arguments as router_forward.
+ */
+int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K,
+                          int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                          int32_t *status, ebl_stream_t stream);
+
+/*
+ * smebu_step -- one SMEBU update of the expert bias, once per optimizer step.
+ * Passage: "SMEBU Load Balancing", "How it works", eqs. (23)-(28).
+ *   nbar = sum_j n_j / N_r
+ *   v_i  = (nbar - n_i) / nbar;  db_i = lambda * tanh(kappa * v_i)
+ *   db_i -= (1/N_r) sum_j db_j      (summed in index order)
+ *   m_i  = beta * m_i + (1 - beta) * db_i;  b_i += m_i
+ * Arithmetic is fp64 with IEEE rounding and no contraction; bias and momentum
+ * are fp32 state, read widened and stored rounded to nearest.
+ *
+ * counts       device, int32 [N_r]: the loads n_i of this step (router_forward output).
+ * bias         device, fp32 [N_r], updated in place.
+ * momentum     device, fp32 [N_r], updated in place (persistent buffer, starts at 0).
+ * lambda, beta, kappa   5e-4, 0.5, 2 in the report.
+ * reset_counts nonzero: counts is zeroed after it is read, ready for the next step.
+ * maxvio_out   device fp32 scalar or NULL: MaxVio = max_i n_i / min_i n_i (+inf if min is 0).
+ * status       device int32 or NULL: EBL_ST_EMPTY_LOAD if sum n = 0 (state untouched).
+ * One CTA; N_r in [1, 256].
+ */
+int smebu_step(int32_t *counts, float *bias, float *momentum, int N_r,
+               float lambda, float beta, float kappa, int reset_counts,
+               float *maxvio_out, int32_t *status, ebl_stream_t stream);
+
+/*
+ * smebu_step_layers -- smebu_step for L independent MoE layers in one launch
+ * (one bias and momentum vector per layer: "SMEBU Load Balancing" writes b as
+ * a vector in R^{N_r} per layer).  counts, bias, momentum are [L, N_r];
+ * maxvio_out is [L] or NULL.  linear != 0 selects the linear, unclamped
+ * ablation db_i = lambda * v_i ("Arcee Trinity Large Technical Report" 2.3;
+ * "SMEBU Load Balancing", last paragraph of "How it works"); kappa is then
+ * ignored.  One CTA per layer.
+ */
+int smebu_step_layers(int32_t *counts, float *bias, float *momentum, int L, int N_r,
+                      float lambda, float beta, float kappa, int linear, int reset_counts,
+                      float *maxvio_out, int32_t *status, ebl_stream_t stream);
+
+/*
+ * sign_update_step -- the aux-loss-free sign update used for the smaller models.
+ * Passage: "SMEBU Load Balancing", eqs. (20)-(22).
+ *   db_i = gamma * sign(nbar - n_i)   (sign(0) = 0)
+ *   b'_i = b_i + db_i;  b_i = b'_i - (1/N_r) sum_j b'_j   (re-centred after the add)
+ * fp64 arithmetic on fp32 state.  Arguments as smebu_step.
+ */
+int sign_update_step(int32_t *counts, float *bias, int N_r, float gamma, int reset_counts,
+                     float *maxvio_out, int32_t *status, ebl_stream_t stream);
+
+/*
+ * moe_dispatch -- expert-sorted, deterministic token dispatch.
+ * The pages name expert parallelism but give no mechanism; this is the plain
+ * stable counting sort of the (token, slot) pairs by expert.
+ *   pairs p = t*K + k, expert e = topk_idx[t,k]
+ *   offsets[0] = 0, offsets[e+1] = offsets[e] + n_e                (int32 [N_r+1])
+ *   j = offsets[e] + #{p' < p : topk_idx flat[p'] == e}             (stable, by p)
+ *   perm[j] = t;  dest[p] = j;  dispatched[j, :] = hidden[t, :]     (bit copy)
+ *
+ * hidden       device, bf16 [T, d], 16-byte aligned, d % 8 == 0.
+ * topk_idx     device, int32 [T, K].
+ * tile_counts  device int32 [ceil(T/128), N_r] from the same router pass, or
+ *              NULL (the per-tile histogram is then computed here).
+ * offsets      device int32 [N_r + 1]; perm, dest device int32 [T*K];
+ * dispatched   device bf16 [T*K, d], 16-byte aligned.
+ * workspace    device scratch of at least ebl_dispatch_workspace_bytes(T, N_r)
+ *              bytes, 16-byte aligned; contents on entry are ignored.
+ * status       EBL_ST_BAD_EXPERT if an id is outside [0, N_r): that pair is
+ *              skipped and its dest is -1.
+ * T*K <= 2^31 - 1.
+ */
+size_t ebl_dispatch_workspace_bytes(int T, int N_r);
+int moe_dispatch(const uint16_t *hidden, const int32_t *topk_idx, const int32_t *tile_counts,
+                 int T, int d, int N_r, int K,
+                 int32_t *offsets, int32_t *perm, int32_t *dest, uint16_t *dispatched,
+                 void *workspace, size_t workspace_bytes, int32_t *status, ebl_stream_t stream);
+
+/*
+ * moe_combine -- gate-weighted un-permute of the expert outputs.
+ *   out[t, :] = sum_{k=0..K-1} gates[t,k] * expert_out[dest[t*K+k], :]
+ * accumulated in fp32 in slot order as acc = fmaf(g, (float)y, acc) from 0,
+ * so the result is deterministic (no atomics) and bit-reproducible.
+ *
+ * expert_out   device, bf16 [T*K, d], 16-byte aligned, d % 8 == 0.
+ * gates        device, fp32 [T, K];  dest device, int32 [T*K] (moe_dispatch output).
+ * out          device, fp32 [T, d], 16-byte aligned, overwritten.
+ * status       EBL_ST_BAD_DEST if a dest is outside [0, T*K): that slot adds nothing.
+ */
+int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *dest,
+                int T, int d, int K, float *out, int32_t *status, ebl_stream_t stream);
+
+/*
+ * ebl_read_internal_status -- copy the library-owned status word (used when a
+ * call passed status == NULL) of the current device to *out, and clear it if
+ * `clear` is nonzero.  Synchronous (waits for the device).
+ */
+int ebl_read_internal_status(int32_t *out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EBL_H */

@@ -1,0 +1,107 @@
+"""Full-size workloads in the launch configuration the benchmark times,
+checked on sampled rows against the oracle and on properties that hold at any
+size (the oracle cannot redo a billion-row GEMM in a test)."""
+import numpy as np
+import pytest
+import torch
+
+import expert_bias_load_b200 as ebl
+import oracle
+import synth
+from tests.parity import assert_gemm_parity, to_np
+
+pytestmark = pytest.mark.gpu
+
+SAMPLE_ROWS = 2048
+
+
+def _sampled_parity(h_dev, W, bias, K, idx, gates, seed):
+    T = h_dev.shape[0]
+    g = torch.Generator().manual_seed(seed)
+    rows = torch.randperm(T, generator=g)[:SAMPLE_ROWS]
+    rows = torch.cat([rows, torch.tensor([0, T - 1])]).sort().values
+    hs = h_dev[rows.to(h_dev.device)].cpu()
+    ref = oracle.router_gemm(hs, W.cpu(), bias.cpu().numpy(), K)
+    r = rows.numpy()
+    return assert_gemm_parity(to_np(idx)[r], to_np(gates)[r], ref, W.shape[0])
+
+
+@pytest.mark.parametrize("name", ["mid", "drift", "ties"])
+def test_router_full_size_sampled(cuda_device, name):
+    cfg = synth.WORKLOADS[name]
+    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
+    dev = cuda_device
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    seed = synth.step_seed(name, 0)
+    if name == "drift":
+        h = synth.hidden_drift(T, d, W, seed=seed, mu=2.0, device=dev)
+    else:
+        h = synth.hidden_normal(T, d, seed=seed, device=dev, quant8=(name == "ties"))
+    bias = synth.dead_start_bias(Nr, device=dev) if name == "ties" else torch.zeros(Nr, device=dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    idx, gates = ebl.router_forward(h, W, bias, K, counts, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    _sampled_parity(h, W, bias, K, idx, gates, seed=T)
+    # properties over all T rows
+    hist = torch.bincount(idx.view(-1).long(), minlength=Nr)
+    assert torch.equal(hist.to(torch.int32), counts)
+    assert int(counts.sum().item()) == T * K
+    srt = idx.sort(dim=1).values
+    assert bool((srt[:, 1:] != srt[:, :-1]).all()) if K > 1 else True      # distinct experts per token
+    gs = gates.double().sum(1)
+    assert float((gs - 1).abs().max()) < K * 2e-7
+    assert bool((gates > 0).all())
+    if name == "ties":
+        assert int(counts[:8].sum().item()) == 0     # bias -1 keeps the 8 dead-start experts out
+
+
+def test_logits_mode_full_tie_workload(cuda_device):
+    """The tie workload in logits mode at full size: bit-exact against the oracle."""
+    cfg = synth.WORKLOADS["ties"]
+    T, Nr, K = cfg["T"], cfg["Nr"], cfg["K"]
+    dev = cuda_device
+    x = synth.logits_normal(T, Nr, seed=synth.step_seed("ties", 1), quant8=True, device=dev)
+    bias = synth.dead_start_bias(Nr, device=dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tiles = torch.empty(((T + 127) // 128, Nr), dtype=torch.int32, device=dev)
+    idx, gates = ebl.router_forward_logits(x, bias, K, counts, tile_counts=tiles)
+    torch.cuda.synchronize()
+    ref = oracle.router_logits(to_np(x), to_np(bias), K, tile_tokens=128)
+    assert np.array_equal(to_np(idx), ref.idx)
+    assert np.array_equal(to_np(gates), ref.gates)
+    assert np.array_equal(to_np(counts), ref.counts)
+    assert np.array_equal(to_np(tiles), ref.tile_counts)
+
+
+def test_dispatch_combine_full_size(cuda_device):
+    """The dispatch workload: router, dispatch, identity expert, combine."""
+    cfg = synth.WORKLOADS["dispatch"]
+    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
+    dev = cuda_device
+    h = synth.hidden_normal(T, d, seed=synth.step_seed("dispatch", 0), device=dev)
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tiles = torch.empty(((T + 127) // 128, Nr), dtype=torch.int32, device=dev)
+    idx, gates = ebl.router_forward(h, W, torch.zeros(Nr, device=dev), K, counts, tile_counts=tiles)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    offsets, perm, dest, X = ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles, status=st)
+    torch.cuda.synchronize()
+    o_off, o_perm, o_dest = oracle.dispatch(to_np(idx), Nr)
+    assert int(st.item()) == 0
+    assert np.array_equal(to_np(offsets), o_off)
+    assert np.array_equal(to_np(perm), o_perm)
+    assert np.array_equal(to_np(dest), o_dest)
+    assert torch.equal(X, h[perm.long()])                       # every row, bit for bit
+    out = ebl.moe_combine(X, gates, dest, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    # sampled rows against the oracle's fp32 chain, all rows against the identity
+    rows = torch.randperm(T, generator=torch.Generator().manual_seed(3))[:256].sort().values
+    pr = (rows[:, None] * K + torch.arange(K)[None, :]).reshape(-1)
+    Xs = to_np(X[dest[pr.to(dev)].long()].view(torch.int16)).view(np.uint16)
+    _, o32 = oracle.combine(Xs, to_np(gates[rows.to(dev)]), np.arange(pr.numel(), dtype=np.int32))
+    assert np.array_equal(to_np(out[rows.to(dev)]), o32)
+    rel = ((out - h.float()).abs() / h.float().abs().clamp_min(1e-30)).max()
+    assert float(rel) <= (2 * K + 1) * 2.0 ** -24

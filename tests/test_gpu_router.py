@@ -1,0 +1,143 @@
+"""Router kernels against the oracle on a B200 (GEMM mode and logits mode)."""
+import numpy as np
+import pytest
+import torch
+
+import expert_bias_load_b200 as ebl
+import oracle
+import synth
+from tests.parity import STATE_RTOL, assert_gemm_parity, rel_err, tile_hist, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_logits(logits, bias, K, want_tiles=True):
+    dev = torch.device("cuda:0")
+    T, Nr = logits.shape
+    x = logits.to(dev)
+    b = bias.to(dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tiles = torch.full(((T + 127) // 128, Nr), -7, dtype=torch.int32, device=dev) if want_tiles else None
+    idx, gates = ebl.router_forward_logits(x, b, K, counts, tile_counts=tiles)
+    torch.cuda.synchronize()
+    return to_np(idx), to_np(gates), to_np(counts), (to_np(tiles) if want_tiles else None)
+
+
+LOGITS_CASES = [
+    # T, Nr, K, quantised, bias kind
+    (2048 + 77, 64, 4, False, "small"),
+    (1000, 8, 8, True, "ties"),
+    (1000, 8, 3, True, "ties"),
+    (513, 16, 1, False, "small"),
+    (3000, 256, 4, True, "dead"),
+    (4096, 128, 8, False, "small"),
+    (129, 200, 5, True, "ties"),
+    (1, 33, 2, False, "small"),
+    (127, 256, 7, False, "dead"),
+]
+
+
+@pytest.mark.parametrize("T,Nr,K,quant,bk", LOGITS_CASES)
+def test_logits_mode_bit_exact(cuda_device, T, Nr, K, quant, bk):
+    logits = synth.logits_normal(T, Nr, seed=100 + T + Nr + K, quant8=quant)
+    if bk == "small":
+        bias = torch.randn(Nr, generator=torch.Generator().manual_seed(K)) * 0.01
+    elif bk == "ties":
+        bias = (torch.randint(-2, 3, (Nr,), generator=torch.Generator().manual_seed(K)) * 0.125).float()
+    else:
+        bias = synth.dead_start_bias(Nr, n_dead=min(8, Nr - K))
+    idx, gates, counts, tiles = _run_logits(logits, bias, K)
+    ref = oracle.router_logits(logits.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx)
+    assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
+    assert np.array_equal(counts, ref.counts)
+    assert np.array_equal(tiles, ref.tile_counts)
+
+
+def test_logits_mode_tie_workload_slice(cuda_device):
+    """The tie workload (values on a 1/8 grid, 8 experts starting at -1) on a
+    65536-token slice: exact ties between scores are everywhere."""
+    T, Nr, K = 65536 + 5, 256, 4
+    logits = synth.logits_normal(T, Nr, seed=synth.step_seed("ties", 0), quant8=True)
+    bias = synth.dead_start_bias(Nr)
+    idx, gates, counts, tiles = _run_logits(logits, bias, K)
+    ref = oracle.router_logits(logits.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx)
+    assert np.array_equal(gates, ref.gates)
+    assert np.array_equal(counts, ref.counts)
+    assert np.array_equal(tiles, ref.tile_counts)
+    assert counts[:8].sum() == 0          # the dead-start experts are never picked at step 0
+
+
+def test_logits_mode_bias_forces_expert(cuda_device):
+    T, Nr, K = 999, 64, 4
+    logits = synth.logits_normal(T, Nr, seed=5)
+    bias = torch.zeros(Nr)
+    bias[17] = 10.0
+    idx, gates, counts, _ = _run_logits(logits, bias, K, want_tiles=False)
+    assert np.all(idx[:, 0] == 17) and counts[17] == T
+
+
+GEMM_CASES = [
+    # T, d, Nr, K
+    (2048, 256, 64, 4),          # the tiny workload
+    (2048 + 77, 256, 64, 4),     # ragged tail
+    (3000, 512, 256, 4),
+    (1000, 2048, 128, 8),        # the mid workload's shape, fewer tokens
+    (777, 128, 32, 1),
+    (777, 128, 32, 8),
+    (129, 64, 96, 3),
+    (1, 64, 32, 2),
+    (5000, 3072, 256, 4),        # the drift workload's shape, fewer tokens
+    (300, 4096, 256, 8),
+]
+
+
+@pytest.mark.parametrize("T,d,Nr,K", GEMM_CASES)
+def test_gemm_mode_vs_oracle(cuda_device, T, d, Nr, K):
+    dev = cuda_device
+    h = synth.hidden_normal(T, d, seed=T * 7 + d)
+    W = synth.router_weight(Nr, d, seed=d + Nr)
+    bias = torch.randn(Nr, generator=torch.Generator().manual_seed(3)) * 0.02
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tiles = torch.full(((T + 127) // 128, Nr), -7, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    idx, gates = ebl.router_forward(h.to(dev), W.to(dev), bias.to(dev), K, counts, tile_counts=tiles,
+                                    status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle.router_gemm(h, W, bias.numpy(), K)
+    gi = to_np(idx)
+    assert_gemm_parity(gi, to_np(gates), ref, Nr, gpu_counts=to_np(counts))
+    assert np.array_equal(to_np(tiles), tile_hist(gi, Nr))
+    g = to_np(gates).astype(np.float64)
+    assert np.allclose(g.sum(1), 1.0, atol=K * 2e-7)
+
+
+def test_gemm_mode_tiny_workload_smebu_steps(cuda_device):
+    """The tiny workload end to end: 10 steps of fresh hidden, router, SMEBU."""
+    dev = cuda_device
+    cfg = synth.WORKLOADS["tiny"]
+    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED)
+    b_g = torch.zeros(Nr, device=dev)
+    m_g = torch.zeros(Nr, device=dev)
+    b_o = np.zeros(Nr, np.float32)
+    m_o = np.zeros(Nr, np.float32)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    maxvio = torch.zeros(1, device=dev)
+    for step in range(cfg["steps"]):
+        h = synth.hidden_normal(T, d, seed=synth.step_seed("tiny", step))
+        ref = oracle.router_gemm(h, W, b_o, K)
+        idx, gates = ebl.router_forward(h.to(dev), W.to(dev), b_g, K, counts)
+        torch.cuda.synchronize()
+        n_gpu = to_np(counts).astype(np.int64)
+        assert_gemm_parity(to_np(idx), to_np(gates), ref, Nr, gpu_counts=n_gpu)
+        ebl.smebu_step(counts, b_g, m_g, reset_counts=True, maxvio=maxvio)
+        # open loop: the oracle's SMEBU is fed the GPU's counts
+        oracle.smebu(n_gpu, b_o, m_o)
+        torch.cuda.synchronize()
+        assert rel_err(to_np(b_g), b_o).max() <= STATE_RTOL
+        assert rel_err(to_np(m_g), m_o).max() <= STATE_RTOL
+        assert float(maxvio.item()) == np.float32(oracle.maxvio(n_gpu)[0])
+        assert int(counts.sum().item()) == 0
