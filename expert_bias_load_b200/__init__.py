@@ -52,6 +52,7 @@ SIGNATURES = {
     "sign_update_step": (_I, [_P, _P, _I, _F, _I, _P, _P, _P]),
     "ebl_dispatch_workspace_bytes": (_SZ, [_I, _I]),
     "moe_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_dispatch_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "ebl_read_internal_status": (_I, [_P, _I]),
 }

@@ -201,6 +201,41 @@ int moe_dispatch(const uint16_t *hidden, const int32_t *topk_idx, const int32_t 
                  void *workspace, size_t workspace_bytes, int32_t *status, ebl_stream_t stream);
 
 /*
+ * moe_dispatch_static -- moe_dispatch without a workspace argument; it
+ * allocates nothing.  The pages have no counterpart to this entry point: it
+ * exists for callers that cannot call cudaMalloc to provide the dispatch
+ * scratch, for example a plugin whose host framework owns every device byte
+ * through its own memory pool and gives the plugin no allocator, or a runtime
+ * that forbids device allocation once it has started serving.
+ *
+ * The scratch lives in one library-owned device array of
+ * EBL_DISPATCH_STATIC_SCRATCH_BYTES (4 MiB), which every GPU that loads the
+ * library holds until the process exits.  A problem fits when
+ * ebl_dispatch_workspace_bytes(T, N_r) <= 4 MiB, i.e. T <= 508288 tokens at
+ * N_r = 256 or T <= 2033536 at N_r = 64; larger problems return EBL_EINVAL
+ * and launch nothing (use moe_dispatch with a caller workspace for them).
+ *
+ * All calls share that one array.  Calls whose kernels overlap on the GPU
+ * (different streams, or different host threads on one device) race on it
+ * and corrupt each other's results; serialise them on one stream.  The array
+ * keeps the last call's contents, which the next call overwrites before
+ * reading, so no clearing is needed between calls.
+ *
+ * The first call on each device does a one-time set-up with that device
+ * current (it looks up the array's device address); make that first call
+ * before any stream capture.  The call makes no cudaMalloc, cudaFree or other
+ * allocating call.
+ *
+ * Arguments, outputs and status bits are those of moe_dispatch.  With
+ * status == NULL, device-side error bits go to a library word nobody reads.
+ */
+#define EBL_DISPATCH_STATIC_SCRATCH_BYTES (4u << 20)
+int moe_dispatch_static(const uint16_t *hidden, const int32_t *topk_idx, const int32_t *tile_counts,
+                        int T, int d, int N_r, int K,
+                        int32_t *offsets, int32_t *perm, int32_t *dest, uint16_t *dispatched,
+                        int32_t *status, ebl_stream_t stream);
+
+/*
  * moe_combine -- gate-weighted un-permute of the expert outputs.
  *   out[t, :] = sum_{k=0..K-1} gates[t,k] * expert_out[dest[t*K+k], :]
  * accumulated in fp32 in slot order as acc = fmaf(g, (float)y, acc) from 0,
