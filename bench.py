@@ -39,6 +39,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-full-step", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="tokens per GPU (default: the tie workload's 1,048,576); smaller values are for profiling")
     return ap.parse_args()
 
 
@@ -163,7 +165,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     import synth
-    cfg = synth.WORKLOADS[WORKLOAD]
+    cfg = dict(synth.WORKLOADS[WORKLOAD])
+    if args.tokens > 0:
+        cfg["T"] = args.tokens
     T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
     config = {"workload": "tie workload: T=%d tokens/GPU, d=%d, N_r=%d, K=%d, hidden on a 1/8 grid, "
                           "8 experts at bias -1.0, GEMM mode" % (T, d, Nr, K),
