@@ -132,7 +132,8 @@ int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float
     if ((rc = get_encoder())) return rc;
     CUtensorMap th, tw;
     if ((rc = encode_bf16_2d(&th, hidden, (uint64_t)T, (uint64_t)d, ebl::kTileTokens))) return rc;
-    if ((rc = encode_bf16_2d(&tw, W_router, (uint64_t)N_r, (uint64_t)d, (uint32_t)N_r))) return rc;
+    if ((rc = encode_bf16_2d(&tw, W_router, (uint64_t)N_r, (uint64_t)d, (uint32_t)ebl::router_gemm_w_box_rows(N_r))))
+        return rc;
     cudaError_t e = ebl::launch_router_gemm(th, tw, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts,
                                             status ? status : di.internal_status, di.num_sms,
                                             reinterpret_cast<cudaStream_t>(stream));

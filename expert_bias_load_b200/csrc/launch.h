@@ -15,8 +15,7 @@ constexpr int kMaxExperts = 256;  // N_r limit
 constexpr int kMaxTopK = 8;       // K limit
 
 // router_gemm.cu
-size_t router_gemm_smem_bytes(int Nr, int stages);
-int router_gemm_stages(int Nr);
+int router_gemm_w_box_rows(int Nr);  // rows of W per TMA box (N_r / CTAs per MMA)
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
                                int32_t *tile_counts, int32_t *status, int num_sms, cudaStream_t stream);

@@ -8,18 +8,30 @@
 // with normalized scores; Top-K on score plus bias; gates from the scores
 // without the bias); "SMEBU Load Balancing" eq. (17).
 //
-// Design (one persistent CTA per SM, warp-specialised):
-//   warp 4      TMA producer: 128x64 hidden tile + N_r x 64 W tile per stage,
-//               128-byte swizzle, into a ring of `stages` shared-memory slots.
-//   warp 5      TMEM owner and MMA issuer: tcgen05.mma M=128, N=N_r, K=16,
-//               fp32 accumulator in TMEM, two accumulator buffers so the
-//               epilogue of tile i overlaps the MMAs of tile i+1.
-//   warps 0-3   epilogue: warp q reads TMEM lanes 32q..32q+31 (one token row
-//               per thread) 32 columns at a time, and runs sigmoid, +bias,
-//               Top-K, gates, output stores and a shared-memory histogram.
+// Design (one persistent CTA per SM, warp-specialised; CG = 1 or 2 CTAs per MMA):
+//   TMA warp    streams the 128x64 hidden tile and a (N_r/CG) x 64 slice of W
+//               for each K step (128-byte swizzle) into a ring of shared-memory
+//               stages.  With CG = 2 the two CTAs of a cluster pair form one
+//               256-token tile: each loads its own 128 token rows and half of
+//               W, so W crosses L2 -> SM once per 256 tokens instead of once
+//               per 128 (half the L2 traffic, half the shared-memory fill).
+//   MMA warp    owns TMEM and issues tcgen05.mma (M=128*CG, N=N_r, K=16; with
+//               CG = 2 issued by the even CTA for both) into a double-buffered
+//               fp32 accumulator (2 x N_r columns per CTA), so the epilogue of
+//               tile i overlaps the MMAs of tile i+1.
+//   epilogue    G groups of 4 warps.  Warp w reads TMEM lane quadrant w%4 (one
+//               token row per thread); group g = w/4 owns the experts
+//               [g*N_r/G, (g+1)*N_r/G).  Each thread runs sigmoid, +bias and a
+//               running Top-K over its experts; groups 1..G-1 hand their
+//               sorted partial lists to group 0 through shared memory, and
+//               group 0 merges them, writes indices and gates, and keeps the
+//               load histogram.  Splitting the experts puts G epilogue warps on
+//               every SM sub-partition, which hides the epilogue's latencies.
 // The logits never leave TMEM.  Counts reach global memory with one atomic per
-// expert per CTA at the end; tile_counts with one store per expert per tile.
-// Every pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
+// expert per CTA; tile_counts with one store per expert per tile.  Every
+// pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
+
+#include <cstdlib>
 
 #include "launch.h"
 #include "ptx.cuh"
@@ -30,14 +42,14 @@ namespace {
 
 constexpr int kBlockK = 64;  // hidden elements per stage: one 128-byte swizzle row
 constexpr int kUmmaK = 16;   // K of one kind::f16 MMA
-constexpr int kEpiWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kChunk = 16;   // TMEM columns per epilogue load
 constexpr int kMaxStages = 8;
 constexpr uint32_t kATileBytes = kTileTokens * kBlockK * 2;  // 16 KiB
 
-__host__ __device__ inline uint32_t b_tile_bytes(int Nr) { return (uint32_t)Nr * kBlockK * 2; }
+__host__ __device__ constexpr int threads_of(int G) { return (4 * G + 2) * 32; }
+
+// Bytes of this CTA's slice of W per stage (N_r/CG rows of 128 bytes).
+__host__ __device__ inline uint32_t b_tile_bytes(int Nr, int CG) { return (uint32_t)(Nr / CG) * kBlockK * 2; }
 
 __host__ __device__ inline uint32_t tmem_columns(int Nr) {
     uint32_t need = 2u * (uint32_t)Nr, c = 32;
@@ -45,15 +57,21 @@ __host__ __device__ inline uint32_t tmem_columns(int Nr) {
     return c;
 }
 
-// Byte offset of the small-object region (barriers, flags, bias, histograms).
-__host__ __device__ inline size_t misc_offset(int Nr, int stages) {
-    return (size_t)stages * (kATileBytes + b_tile_bytes(Nr));
-}
+// Shared memory after the stage ring: barriers, then (16-byte aligned) the
+// bias, the histograms and the partial-list exchange buffers.
+struct Misc {
+    size_t bar_off, vec_off, total;
+};
 
-__host__ __device__ inline size_t misc_bytes(int Nr, int stages) {
-    // full[S], empty[S], tfull[2], tempty[2], epi_sync, drain (8 B each);
-    // tmem slot + abort flag + pad (16 B); bias, hist_total, hist_tile[2] (4 Nr each)
-    return (size_t)(2 * stages + 6) * 8 + 16 + (size_t)4 * Nr * 4;
+__host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int CG, int stages) {
+    Misc m;
+    m.bar_off = (size_t)stages * (kATileBytes + b_tile_bytes(Nr, CG));
+    // full[S], empty[S], tfull[2], tempty[2], epi_sync, drain, list_full, list_empty; tmem slot, abort flag
+    const size_t bars = (size_t)(2 * stages + 8) * 8 + 16;
+    m.vec_off = m.bar_off + ((bars + 15) & ~size_t(15));
+    const size_t vec = (size_t)4 * Nr * 4 + (size_t)3 * (G - 1) * K * kTileTokens * 4;
+    m.total = m.vec_off + vec;
+    return m;
 }
 
 __device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t parity) {
@@ -63,63 +81,69 @@ __device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-// tcgen05.wait::ld, with the loaded registers tied to it so that no use of
-// them can be scheduled before the wait.
-__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.wait::ld.sync.aligned;"
-        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-          "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
-          "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
-          "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-          "+r"(r[30]), "+r"(r[31])
-        :
-        : "memory");
-}
-
 template <int K>
-__device__ __forceinline__ void consume_chunk(const uint32_t (&r)[32], const float *__restrict__ bias_s, int c,
+__device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const float *__restrict__ bias_s, int c,
                                               RowTopK<K> &tk) {
+    const float4 *b4 = reinterpret_cast<const float4 *>(bias_s + c);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const float x = __uint_as_float(r[j]);
-        const float s = fast_rcp(1.0f + __expf(-x));
-        const float kv = __fadd_rn(s, bias_s[c + j]);
-        tk.push(kv, s, c + j);
+    for (int q = 0; q < kChunk / 4; ++q) {
+        const float4 bb = b4[q];
+        const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float x = __uint_as_float(r[4 * q + j]);
+            const float s = fast_rcp(1.0f + __expf(-x));
+            tk.push(__fadd_rn(s, bv[j]), s, c + 4 * q + j);
+        }
     }
 }
 
-template <int K>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int K, int G, int CG>
+__global__ void __launch_bounds__(threads_of(G), 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
                        const float *__restrict__ bias, int T, int d, int Nr, int stages,
                        int32_t *__restrict__ topk_idx, float *__restrict__ gates, int32_t *__restrict__ counts,
                        int32_t *__restrict__ tile_counts, int32_t *__restrict__ status) {
+    constexpr int kEpiWarps = 4 * G;
+    constexpr int kProducerWarp = 4 * G;
+    constexpr int kMmaWarp = 4 * G + 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    const uint32_t b_bytes = b_tile_bytes(Nr);
+    const Misc ml = misc_layout(Nr, K, G, CG, stages);
+    const uint32_t b_bytes = b_tile_bytes(Nr, CG);
     uint8_t *smA = smem;
     uint8_t *smB = smem + (size_t)stages * kATileBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + misc_offset(Nr, stages));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ml.bar_off);
     uint64_t *empty = full + stages;
     uint64_t *tfull = empty + stages;
     uint64_t *tempty = tfull + 2;
     uint64_t *epi_sync = tempty + 2;
     uint64_t *drain = epi_sync + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *list_full = drain + 1;
+    uint64_t *list_empty = list_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(list_empty + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *bias_s = reinterpret_cast<float *>(tmem_slot + 4);
+    float *bias_s = reinterpret_cast<float *>(smem + ml.vec_off);
     int *hist_total = reinterpret_cast<int *>(bias_s + Nr);
     int *hist_tile = hist_total + Nr;  // [2][Nr]
+    float *pl_key = reinterpret_cast<float *>(hist_tile + 2 * Nr);  // [G-1][K][128]
+    float *pl_s = pl_key + (G - 1) * K * kTileTokens;
+    int *pl_idx = reinterpret_cast<int *>(pl_s + (G - 1) * K * kTileTokens);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    // With CG = 2, CTA `rank` of a cluster pair owns 128-token tile 2*p + rank
+    // of pair tile p; the even CTA (rank 0) issues the MMAs for both.
+    const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+    const int unit = (int)blockIdx.x / CG;       // cluster index
+    const int num_units = (int)gridDim.x / CG;   // clusters in the grid
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;      // 128-token tiles
+    const int num_work = (num_tiles + CG - 1) / CG;                 // 128*CG-token tiles
     const int num_kb = d / kBlockK;
     const uint32_t tcols = tmem_columns(Nr);
 
-    for (int i = threadIdx.x; i < Nr; i += kThreads) {
+    for (int i = threadIdx.x; i < Nr; i += threads_of(G)) {
         bias_s[i] = bias[i];
         hist_total[i] = 0;
         hist_tile[i] = 0;
@@ -132,21 +156,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], kEpiWarps * 32);
+            mbar_init(&tempty[a], CG * kEpiWarps);  // one arrival per epilogue warp of the pair
         }
-        mbar_init(epi_sync, kEpiWarps * 32);
+        mbar_init(epi_sync, 128);
         mbar_init(drain, 1);
+        mbar_init(list_full, (G - 1) * 128 > 0 ? (G - 1) * 128 : 1);
+        mbar_init(list_empty, 128);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_h);
         prefetch_tmap(&tmap_w);
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, tcols);
-        tmem_relinquish();
+        if constexpr (CG == 2) {
+            tmem_alloc_pair(tmem_slot, tcols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, tcols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -154,20 +186,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol_h = l2_policy_evict_first();  // hidden: read once
             const uint64_t pol_w = l2_policy_evict_last();   // W_router: re-read by every tile
+            const int w_row0 = (int)rank * (Nr / CG);        // this CTA's slice of W
             int s = 0;
             uint32_t ph = 0;
-            uint32_t issued = 0, issued_ph = 0;  // per stage: ever issued, parity of last issue
+            uint32_t issued = 0, issued_ph = 0;  // per stage: ever issued, parity of the last issue
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int wk = unit; wk < num_work && ok; wk += num_units) {
+                const int tile = wk * CG + (int)rank;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], kATileBytes + b_bytes);
-                    tma_load_2d(smA + (size_t)s * kATileBytes, &tmap_h, &full[s], kb * kBlockK, tile * kTileTokens,
-                                pol_h);
-                    tma_load_2d(smB + (size_t)s * b_bytes, &tmap_w, &full[s], kb * kBlockK, 0, pol_w);
+                    if constexpr (CG == 2) {
+                        // both CTAs' loads complete on the even CTA's barrier, which
+                        // the even CTA arms with the bytes of the whole pair
+                        const uint32_t bar0 = map_to_cta(smem_u32(&full[s]), 0);
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (kATileBytes + b_bytes));
+                        tma_load_2d_pair(smA + (size_t)s * kATileBytes, &tmap_h, bar0, kb * kBlockK,
+                                         tile * kTileTokens, pol_h);
+                        tma_load_2d_pair(smB + (size_t)s * b_bytes, &tmap_w, bar0, kb * kBlockK, w_row0, pol_w);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], kATileBytes + b_bytes);
+                        tma_load_2d(smA + (size_t)s * kATileBytes, &tmap_h, &full[s], kb * kBlockK,
+                                    tile * kTileTokens, pol_h);
+                        tma_load_2d(smB + (size_t)s * b_bytes, &tmap_w, &full[s], kb * kBlockK, 0, pol_w);
+                    }
                     issued |= 1u << s;
                     issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == stages) {
@@ -179,19 +223,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) {
                 atomicOr(status, kStTimeout);
                 *abort_flag = 1;
-                // let the loads already in flight land before the CTA exits
-                for (int t = 0; t < stages; ++t)
-                    if (issued & (1u << t)) wait_timed(&full[t], (issued_ph >> t) & 1u);
+                if constexpr (CG == 2) {
+                    // the pair's loads signal the even CTA: give in-flight loads a
+                    // fixed grace period to land instead of waiting on a barrier
+                    const uint64_t t0 = global_timer_ns();
+                    while (global_timer_ns() - t0 < 2000000ull) {
+                    }
+                } else {
+                    for (int t = 0; t < stages; ++t)
+                        if (issued & (1u << t)) wait_timed(&full[t], (issued_ph >> t) & 1u);
+                }
             }
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kTileTokens, (uint32_t)Nr);
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(kTileTokens * CG, (uint32_t)Nr);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
             int it = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+            for (int wk = unit; wk < num_work && ok; wk += num_units, ++it) {
                 const int acc = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
                 if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u, abort_flag)) {
@@ -210,34 +261,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b0 = smem_u32(smB + (size_t)s * b_bytes);
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
-                        umma_bf16(d_tmem, smem_desc_sw128_kmajor(a0 + kk * kUmmaK * 2),
-                                  smem_desc_sw128_kmajor(b0 + kk * kUmmaK * 2), idesc, (uint32_t)(kb | kk));
+                        const uint64_t ad = smem_desc_sw128_kmajor(a0 + kk * kUmmaK * 2);
+                        const uint64_t bd = smem_desc_sw128_kmajor(b0 + kk * kUmmaK * 2);
+                        if constexpr (CG == 2)
+                            umma_bf16_pair(d_tmem, ad, bd, idesc, (uint32_t)(kb | kk));
+                        else
+                            umma_bf16(d_tmem, ad, bd, idesc, (uint32_t)(kb | kk));
                     }
-                    umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+                    // free the stage (in both CTAs) once these MMAs have read it
+                    if constexpr (CG == 2)
+                        umma_commit_pair_mc(&empty[s], 0x3);
+                    else
+                        umma_commit(&empty[s]);
                     if (++s == stages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[acc]);  // accumulator complete
+                // accumulator complete (in both CTAs)
+                if constexpr (CG == 2)
+                    umma_commit_pair_mc(&tfull[acc], 0x3);
+                else
+                    umma_commit(&tfull[acc]);
             }
             if (!ok) {
                 atomicOr(status, kStTimeout);
                 *abort_flag = 1;
             }
             // every MMA this thread issued has finished once `drain` completes
-            umma_commit(drain);
+            if constexpr (CG == 2)
+                umma_commit_pair(drain);
+            else
+                umma_commit(drain);
             wait_timed(drain, 0);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int quad = warp & 3;
+        const int group = warp >> 2;
+        const int rloc = quad * 32 + lane;  // row within the tile = TMEM lane
+        const int cpg = Nr / G;             // experts per group (a multiple of 32)
+        const int c0 = group * cpg;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const bool want_tiles = tile_counts != nullptr;
         uint32_t sync_ph = 0;
         bool ok = true;
         int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        for (int wk = unit; wk < num_work; wk += num_units, ++it) {
+            const int tile = wk * CG + (int)rank;
             const int acc = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) {
@@ -248,31 +320,71 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             RowTopK<K> tk;
             tk.init();
-            const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * Nr);
-            uint32_t ra[32], rb[32];
+            const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * Nr + c0);
+            uint32_t ra[kChunk], rb[kChunk];
             __syncwarp();
-            tmem_ld_32x32b_x32(taddr, ra);
-            tmem_ld_wait_regs(ra);
-            for (int c = 0; c < Nr; c += 64) {
-                const bool has_b = c + 32 < Nr;
+            tmem_ld_32x32b_x16(taddr, ra);
+            tmem_ld_wait_x16(ra);
+            for (int c = 0; c < cpg; c += 2 * kChunk) {  // cpg % 32 == 0: chunks come in pairs
                 __syncwarp();
-                if (has_b) tmem_ld_32x32b_x32(taddr + (uint32_t)(c + 32), rb);
-                consume_chunk<K>(ra, bias_s, c, tk);
-                if (has_b) {
-                    __syncwarp();
-                    tmem_ld_wait_regs(rb);
-                    const bool has_a = c + 64 < Nr;
-                    if (has_a) tmem_ld_32x32b_x32(taddr + (uint32_t)(c + 64), ra);
-                    consume_chunk<K>(rb, bias_s, c + 32, tk);
-                    __syncwarp();
-                    if (has_a) tmem_ld_wait_regs(ra);
-                }
+                tmem_ld_32x32b_x16(taddr + (uint32_t)(c + kChunk), rb);
+                consume_chunk<K>(ra, bias_s, c0 + c, tk);
+                __syncwarp();
+                tmem_ld_wait_x16(rb);
+                const bool more = c + 2 * kChunk < cpg;
+                if (more) tmem_ld_32x32b_x16(taddr + (uint32_t)(c + 2 * kChunk), ra);
+                consume_chunk<K>(rb, bias_s, c0 + c + kChunk, tk);
+                __syncwarp();
+                if (more) tmem_ld_wait_x16(ra);
             }
-            // accumulator fully read: hand it back to the MMA warp
+            // this warp is done with the accumulator: hand it back to the MMA warp
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 2)
+                    mbar_arrive_cluster(map_to_cta(smem_u32(&tempty[acc]), 0));
+                else
+                    mbar_arrive(&tempty[acc]);
+            }
 
-            const int row = tile * kTileTokens + warp * 32 + lane;
+            if (group > 0) {
+                // publish the sorted partial list for group 0
+                if (!mbar_wait(list_empty, (uint32_t)(it & 1) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int base = (group - 1) * K * kTileTokens + rloc;
+#pragma unroll
+                for (int k = 0; k < K; ++k) {
+                    pl_key[base + k * kTileTokens] = tk.key[k];
+                    pl_s[base + k * kTileTokens] = tk.score[k];
+                    pl_idx[base + k * kTileTokens] = tk.idx[k];
+                }
+                mbar_arrive(list_full);
+                continue;
+            }
+
+            if (G > 1) {
+                // merge the partial lists in group order: every expert of a later
+                // group has a higher index, and each list is sorted by (key desc,
+                // index asc), so pushes keep the tie rule
+                if (!mbar_wait(list_full, (uint32_t)(it & 1), abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                for (int g = 1; g < G; ++g) {
+                    const int base = (g - 1) * K * kTileTokens + rloc;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        const float kv = pl_key[base + k * kTileTokens];
+                        if (!(kv > tk.key[K - 1])) break;
+                        tk.push(kv, pl_s[base + k * kTileTokens], pl_idx[base + k * kTileTokens]);
+                    }
+                }
+                mbar_arrive(list_empty);
+            }
+
+            const int row = tile * kTileTokens + rloc;
             int *hist = want_tiles ? hist_tile + (it & 1) * Nr : hist_total;
             if (row < T) {
                 float sum = 0.0f;
@@ -308,22 +420,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 sync_ph ^= 1u;
-                for (int e = threadIdx.x; e < Nr; e += kEpiWarps * 32) {
+                const bool real_tile = tile < num_tiles;  // a pair's odd tile can lie past T
+                for (int e = rloc; e < Nr; e += 128) {
                     const int v = hist[e];
-                    tile_counts[(size_t)tile * Nr + e] = v;
+                    if (real_tile) tile_counts[(size_t)tile * Nr + e] = v;
                     hist_total[e] += v;
                     hist[e] = 0;
                 }
             }
         }
-        if (ok) {
-            mbar_arrive(epi_sync);
-            ok = mbar_wait(epi_sync, sync_ph, abort_flag);
+        if (group == 0) {
+            if (ok) {
+                mbar_arrive(epi_sync);
+                ok = mbar_wait(epi_sync, sync_ph, abort_flag);
+            }
+            if (ok) {
+                for (int e = rloc; e < Nr; e += 128)
+                    if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
+            }
         }
-        if (ok) {
-            for (int e = threadIdx.x; e < Nr; e += kEpiWarps * 32)
-                if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
-        } else {
+        if (!ok) {
             atomicOr(status, kStTimeout);
             *abort_flag = 1;
         }
@@ -331,40 +447,97 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync();  // neither CTA leaves while the pair may still touch it
     if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, tcols);
+        if constexpr (CG == 2)
+            tmem_dealloc_pair(tmem_base, tcols);
+        else
+            tmem_dealloc(tmem_base, tcols);
     }
+}
+
+int groups_for(int Nr) { return (Nr % 128 == 0) ? 4 : ((Nr % 64 == 0) ? 2 : 1); }
+
+// CTAs per MMA: 2 (pair) by default; EBL_ROUTER_CTA_GROUP=1 selects single-CTA tiles.
+int cta_group() {
+    static int cg = [] {
+        const char *e = getenv("EBL_ROUTER_CTA_GROUP");
+        return (e && e[0] == '1') ? 1 : 2;
+    }();
+    return cg;
+}
+
+int stages_for(int Nr, int K, int G, int CG) {
+    const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
+    int s = kMaxStages;
+    while (s > 2 && 1024 + misc_layout(Nr, K, G, CG, s).total > budget) --s;
+    return s;
+}
+
+template <int K, int G, int CG>
+cudaError_t launch_kgc(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
+                       int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
+                       int num_sms, cudaStream_t stream) {
+    auto kern = router_gemm_kernel<K, G, CG>;
+    const int stages = stages_for(Nr, K, G, CG);
+    const size_t smem = 1024 + misc_layout(Nr, K, G, CG, stages).total;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    const int num_work = (num_tiles + CG - 1) / CG;
+    int units = num_sms / CG;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(threads_of(G), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    if (CG == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(2 * units, 1, 1);
+        int active = 0;  // clusters that fit on the device at once
+        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 && active < units)
+            units = active;
+        (void)cudaGetLastError();
+    }
+    if (units > num_work) units = num_work;
+    cfg.gridDim = dim3(CG * units, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, status);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
+
+template <int K, int G>
+cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
+                      int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
+                      int num_sms, cudaStream_t stream) {
+    if (cta_group() == 2)
+        return launch_kgc<K, G, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+    return launch_kgc<K, G, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
 }
 
 template <int K>
 cudaError_t launch_k(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
                      int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
                      int num_sms, cudaStream_t stream) {
-    const int stages = router_gemm_stages(Nr);
-    const size_t smem = router_gemm_smem_bytes(Nr, stages);
-    cudaError_t err =
-        cudaFuncSetAttribute(router_gemm_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
-    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
-    router_gemm_kernel<K><<<grid, kThreads, smem, stream>>>(th, tw, bias, T, d, Nr, stages, idx, gates, counts,
-                                                           tile_counts, status);
-    return cudaGetLastError();
+    switch (groups_for(Nr)) {
+        case 4:
+            return launch_kg<K, 4>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+        case 2:
+            return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+        default:
+            return launch_kg<K, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+    }
 }
 
 }  // namespace
 
-int router_gemm_stages(int Nr) {
-    const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
-    int s = kMaxStages;
-    while (s > 2 && router_gemm_smem_bytes(Nr, s) > budget) --s;
-    return s;
-}
-
-size_t router_gemm_smem_bytes(int Nr, int stages) {
-    return 1024 /* alignment slack */ + misc_offset(Nr, stages) + misc_bytes(Nr, stages);
-}
+int router_gemm_w_box_rows(int Nr) { return Nr / cta_group(); }
 
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
