@@ -8,15 +8,17 @@
 // with normalized scores; Top-K on score plus bias; gates from the scores
 // without the bias); "SMEBU Load Balancing" eq. (17).
 //
-// Design (one persistent CTA per SM, warp-specialised; CG = 1 or 2 CTAs per MMA):
-//   TMA warp    streams the 128x64 hidden tile and a (N_r/CG) x 64 slice of W
-//               for each K step (128-byte swizzle) into a ring of shared-memory
-//               stages.  With CG = 2 the two CTAs of a cluster pair form one
-//               256-token tile: each loads its own 128 token rows and half of
-//               W, so W crosses L2 -> SM once per 256 tokens instead of once
-//               per 128 (half the L2 traffic, half the shared-memory fill).
-//   MMA warp    owns TMEM and issues tcgen05.mma (M=128*CG, N=N_r, K=16; with
-//               CG = 2 issued by the even CTA for both) into a double-buffered
+// Design (one persistent CTA per SM, warp-specialised, CTA pairs):
+//   pairs       the two CTAs of a 2-CTA cluster form one 256-token tile: each
+//               loads its own 128 token rows and half of W, and one
+//               tcgen05.mma.cta_group::2 (M=256) covers both, so W crosses
+//               L2 -> SM once per 256 tokens (half the L2 traffic and half the
+//               shared-memory fill of single-CTA tiles).
+//   TMA warp    streams the 128x128 hidden tile and the (N_r/2) x 128 slice of W
+//               for each K step (two 64-column boxes each, 128-byte swizzle)
+//               into a ring of shared-memory stages.
+//   MMA warp    owns TMEM; in the even CTA it issues tcgen05.mma (M=256, N=N_r,
+//               K=16, 8 per stage) for the pair into a double-buffered
 //               fp32 accumulator (2 x N_r columns per CTA), so the epilogue of
 //               tile i overlaps the MMAs of tile i+1.
 //   epilogue    G groups of 4 warps.  Warp w reads TMEM lane quadrant w%4 (one
@@ -31,8 +33,6 @@
 // expert per CTA; tile_counts with one store per expert per tile.  Every
 // pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
 
-#include <cstdlib>
-
 #include "launch.h"
 #include "ptx.cuh"
 #include "topk.cuh"
@@ -40,16 +40,22 @@
 namespace ebl {
 namespace {
 
-constexpr int kBlockK = 64;  // hidden elements per stage: one 128-byte swizzle row
+constexpr int kSubK = 64;                // hidden elements per TMA box: one 128-byte swizzle row
+constexpr int kNSub = 2;                 // boxes per pipeline stage
+constexpr int kBlockK = kSubK * kNSub;   // hidden elements per stage (8 MMAs between barriers)
 constexpr int kUmmaK = 16;   // K of one kind::f16 MMA
 constexpr int kChunk = 16;   // TMEM columns per epilogue load
 constexpr int kMaxStages = 8;
-constexpr uint32_t kATileBytes = kTileTokens * kBlockK * 2;  // 16 KiB
+constexpr uint32_t kASubBytes = kTileTokens * kSubK * 2;
+constexpr uint32_t kATileBytes = kASubBytes * kNSub;
 
 __host__ __device__ constexpr int threads_of(int G) { return (4 * G + 2) * 32; }
 
-// Bytes of this CTA's slice of W per stage (N_r/CG rows of 128 bytes).
-__host__ __device__ inline uint32_t b_tile_bytes(int Nr, int CG) { return (uint32_t)(Nr / CG) * kBlockK * 2; }
+constexpr int kPair = 2;  // CTAs per MMA (cluster size)
+
+// Bytes of this CTA's slice of W per box and per stage (N_r/2 rows of 128 bytes).
+__host__ __device__ inline uint32_t b_sub_bytes(int Nr) { return (uint32_t)(Nr / kPair) * kSubK * 2; }
+__host__ __device__ inline uint32_t b_tile_bytes(int Nr) { return b_sub_bytes(Nr) * kNSub; }
 
 __host__ __device__ inline uint32_t tmem_columns(int Nr) {
     uint32_t need = 2u * (uint32_t)Nr, c = 32;
@@ -63,9 +69,9 @@ struct Misc {
     size_t bar_off, vec_off, total;
 };
 
-__host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int CG, int stages) {
+__host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int stages) {
     Misc m;
-    m.bar_off = (size_t)stages * (kATileBytes + b_tile_bytes(Nr, CG));
+    m.bar_off = (size_t)stages * (kATileBytes + b_tile_bytes(Nr));
     // full[S], empty[S], tfull[2], tempty[2], epi_sync, drain, list_full, list_empty; tmem slot, abort flag
     const size_t bars = (size_t)(2 * stages + 8) * 8 + 16;
     m.vec_off = m.bar_off + ((bars + 15) & ~size_t(15));
@@ -98,7 +104,7 @@ __device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const
     }
 }
 
-template <int K, int G, int CG>
+template <int K, int G>
 __global__ void __launch_bounds__(threads_of(G), 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
                        const float *__restrict__ bias, int T, int d, int Nr, int stages,
@@ -110,8 +116,8 @@ __global__ void __launch_bounds__(threads_of(G), 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    const Misc ml = misc_layout(Nr, K, G, CG, stages);
-    const uint32_t b_bytes = b_tile_bytes(Nr, CG);
+    const Misc ml = misc_layout(Nr, K, G, stages);
+    const uint32_t b_bytes = b_tile_bytes(Nr);
     uint8_t *smA = smem;
     uint8_t *smB = smem + (size_t)stages * kATileBytes;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + ml.bar_off);
@@ -133,14 +139,14 @@ __global__ void __launch_bounds__(threads_of(G), 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // With CG = 2, CTA `rank` of a cluster pair owns 128-token tile 2*p + rank
-    // of pair tile p; the even CTA (rank 0) issues the MMAs for both.
-    const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
-    const int unit = (int)blockIdx.x / CG;       // cluster index
-    const int num_units = (int)gridDim.x / CG;   // clusters in the grid
-    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;      // 128-token tiles
-    const int num_work = (num_tiles + CG - 1) / CG;                 // 128*CG-token tiles
-    const int num_kb = d / kBlockK;
+    // CTA `rank` of a cluster pair owns 128-token tile 2*p + rank of pair
+    // tile p; the even CTA (rank 0) issues the MMAs for both.
+    const uint32_t rank = cluster_ctarank();
+    const int unit = (int)blockIdx.x / kPair;       // cluster index
+    const int num_units = (int)gridDim.x / kPair;   // clusters in the grid
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;   // 128-token tiles
+    const int num_work = (num_tiles + kPair - 1) / kPair;        // 256-token pair tiles
+    const int num_kb = (d + kBlockK - 1) / kBlockK;  // a last half stage reads zeros past d
     const uint32_t tcols = tmem_columns(Nr);
 
     for (int i = threadIdx.x; i < Nr; i += threads_of(G)) {
@@ -156,7 +162,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], CG * kEpiWarps);  // one arrival per epilogue warp of the pair
+            mbar_init(&tempty[a], kPair * kEpiWarps);  // one arrival per epilogue warp of the pair
         }
         mbar_init(epi_sync, 128);
         mbar_init(drain, 1);
@@ -167,18 +173,13 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         prefetch_tmap(&tmap_h);
         prefetch_tmap(&tmap_w);
     }
-    if (warp == kMmaWarp) {
-        if constexpr (CG == 2) {
-            tmem_alloc_pair(tmem_slot, tcols);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(tmem_slot, tcols);
-            tmem_relinquish();
-        }
+    if (warp == kMmaWarp) {  // same warp id in both CTAs, as the pair allocation requires
+        tmem_alloc_pair(tmem_slot, tcols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
+    cluster_sync();  // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -186,34 +187,27 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         if (lane == 0) {
             const uint64_t pol_h = l2_policy_evict_first();  // hidden: read once
             const uint64_t pol_w = l2_policy_evict_last();   // W_router: re-read by every tile
-            const int w_row0 = (int)rank * (Nr / CG);        // this CTA's slice of W
+            const int w_row0 = (int)rank * (Nr / kPair);     // this CTA's slice of W
             int s = 0;
             uint32_t ph = 0;
-            uint32_t issued = 0, issued_ph = 0;  // per stage: ever issued, parity of the last issue
             bool ok = true;
             for (int wk = unit; wk < num_work && ok; wk += num_units) {
-                const int tile = wk * CG + (int)rank;
+                const int tile = wk * kPair + (int)rank;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if constexpr (CG == 2) {
-                        // both CTAs' loads complete on the even CTA's barrier, which
-                        // the even CTA arms with the bytes of the whole pair
-                        const uint32_t bar0 = map_to_cta(smem_u32(&full[s]), 0);
-                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (kATileBytes + b_bytes));
-                        tma_load_2d_pair(smA + (size_t)s * kATileBytes, &tmap_h, bar0, kb * kBlockK,
-                                         tile * kTileTokens, pol_h);
-                        tma_load_2d_pair(smB + (size_t)s * b_bytes, &tmap_w, bar0, kb * kBlockK, w_row0, pol_w);
-                    } else {
-                        mbar_arrive_expect_tx(&full[s], kATileBytes + b_bytes);
-                        tma_load_2d(smA + (size_t)s * kATileBytes, &tmap_h, &full[s], kb * kBlockK,
-                                    tile * kTileTokens, pol_h);
-                        tma_load_2d(smB + (size_t)s * b_bytes, &tmap_w, &full[s], kb * kBlockK, 0, pol_w);
+                    // both CTAs' loads complete on the even CTA's barrier, which the
+                    // even CTA arms with the bytes of the whole pair
+                    const uint32_t bar0 = map_to_cta(smem_u32(&full[s]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)kPair * (kATileBytes + b_bytes));
+                    for (int u = 0; u < kNSub; ++u) {
+                        tma_load_2d_pair(smA + (size_t)s * kATileBytes + u * kASubBytes, &tmap_h, bar0,
+                                         kb * kBlockK + u * kSubK, tile * kTileTokens, pol_h);
+                        tma_load_2d_pair(smB + (size_t)s * b_bytes + u * b_sub_bytes(Nr), &tmap_w, bar0,
+                                         kb * kBlockK + u * kSubK, w_row0, pol_w);
                     }
-                    issued |= 1u << s;
-                    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
                     if (++s == stages) {
                         s = 0;
                         ph ^= 1u;
@@ -223,21 +217,16 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             if (!ok) {
                 atomicOr(status, kStTimeout);
                 *abort_flag = 1;
-                if constexpr (CG == 2) {
-                    // the pair's loads signal the even CTA: give in-flight loads a
-                    // fixed grace period to land instead of waiting on a barrier
-                    const uint64_t t0 = global_timer_ns();
-                    while (global_timer_ns() - t0 < 2000000ull) {
-                    }
-                } else {
-                    for (int t = 0; t < stages; ++t)
-                        if (issued & (1u << t)) wait_timed(&full[t], (issued_ph >> t) & 1u);
+                // the pair's loads signal the even CTA: give loads in flight a
+                // fixed grace period to land instead of waiting on a barrier
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 2000000ull) {
                 }
             }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kTileTokens * CG, (uint32_t)Nr);
+            const uint32_t idesc = idesc_bf16_f32(kTileTokens * kPair, (uint32_t)Nr);
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -261,18 +250,13 @@ __global__ void __launch_bounds__(threads_of(G), 1)
                     const uint32_t b0 = smem_u32(smB + (size_t)s * b_bytes);
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / kUmmaK; ++kk) {
-                        const uint64_t ad = smem_desc_sw128_kmajor(a0 + kk * kUmmaK * 2);
-                        const uint64_t bd = smem_desc_sw128_kmajor(b0 + kk * kUmmaK * 2);
-                        if constexpr (CG == 2)
-                            umma_bf16_pair(d_tmem, ad, bd, idesc, (uint32_t)(kb | kk));
-                        else
-                            umma_bf16(d_tmem, ad, bd, idesc, (uint32_t)(kb | kk));
+                        const int u = kk / (kSubK / kUmmaK), w = kk % (kSubK / kUmmaK);
+                        const uint64_t ad = smem_desc_sw128_kmajor(a0 + u * kASubBytes + w * kUmmaK * 2);
+                        const uint64_t bd = smem_desc_sw128_kmajor(b0 + u * b_sub_bytes(Nr) + w * kUmmaK * 2);
+                        umma_bf16_pair(d_tmem, ad, bd, idesc, (uint32_t)(kb | kk));
                     }
                     // free the stage (in both CTAs) once these MMAs have read it
-                    if constexpr (CG == 2)
-                        umma_commit_pair_mc(&empty[s], 0x3);
-                    else
-                        umma_commit(&empty[s]);
+                    umma_commit_pair_mc(&empty[s], 0x3);
                     if (++s == stages) {
                         s = 0;
                         ph ^= 1u;
@@ -280,20 +264,14 @@ __global__ void __launch_bounds__(threads_of(G), 1)
                 }
                 if (!ok) break;
                 // accumulator complete (in both CTAs)
-                if constexpr (CG == 2)
-                    umma_commit_pair_mc(&tfull[acc], 0x3);
-                else
-                    umma_commit(&tfull[acc]);
+                umma_commit_pair_mc(&tfull[acc], 0x3);
             }
             if (!ok) {
                 atomicOr(status, kStTimeout);
                 *abort_flag = 1;
             }
             // every MMA this thread issued has finished once `drain` completes
-            if constexpr (CG == 2)
-                umma_commit_pair(drain);
-            else
-                umma_commit(drain);
+            umma_commit_pair(drain);
             wait_timed(drain, 0);
         }
     } else {
@@ -309,7 +287,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         bool ok = true;
         int it = 0;
         for (int wk = unit; wk < num_work; wk += num_units, ++it) {
-            const int tile = wk * CG + (int)rank;
+            const int tile = wk * kPair + (int)rank;
             const int acc = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait(&tfull[acc], use & 1u, abort_flag)) {
@@ -340,12 +318,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             // this warp is done with the accumulator: hand it back to the MMA warp
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                if constexpr (CG == 2)
-                    mbar_arrive_cluster(map_to_cta(smem_u32(&tempty[acc]), 0));
-                else
-                    mbar_arrive(&tempty[acc]);
-            }
+            if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_u32(&tempty[acc]), 0));
 
             if (group > 0) {
                 // publish the sorted partial list for group 0
@@ -447,78 +420,55 @@ __global__ void __launch_bounds__(threads_of(G), 1)
 
     tc_fence_before();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync();  // neither CTA leaves while the pair may still touch it
+    cluster_sync();  // neither CTA leaves while the pair may still touch it
     if (warp == kMmaWarp) {
         tc_fence_after();
-        if constexpr (CG == 2)
-            tmem_dealloc_pair(tmem_base, tcols);
-        else
-            tmem_dealloc(tmem_base, tcols);
+        tmem_dealloc_pair(tmem_base, tcols);
     }
 }
 
 int groups_for(int Nr) { return (Nr % 128 == 0) ? 4 : ((Nr % 64 == 0) ? 2 : 1); }
 
-// CTAs per MMA: 2 (pair) by default; EBL_ROUTER_CTA_GROUP=1 selects single-CTA tiles.
-int cta_group() {
-    static int cg = [] {
-        const char *e = getenv("EBL_ROUTER_CTA_GROUP");
-        return (e && e[0] == '1') ? 1 : 2;
-    }();
-    return cg;
-}
-
-int stages_for(int Nr, int K, int G, int CG) {
+int stages_for(int Nr, int K, int G) {
     const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
     int s = kMaxStages;
-    while (s > 2 && 1024 + misc_layout(Nr, K, G, CG, s).total > budget) --s;
+    while (s > 2 && 1024 + misc_layout(Nr, K, G, s).total > budget) --s;
     return s;
-}
-
-template <int K, int G, int CG>
-cudaError_t launch_kgc(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
-                       int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
-                       int num_sms, cudaStream_t stream) {
-    auto kern = router_gemm_kernel<K, G, CG>;
-    const int stages = stages_for(Nr, K, G, CG);
-    const size_t smem = 1024 + misc_layout(Nr, K, G, CG, stages).total;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
-    const int num_work = (num_tiles + CG - 1) / CG;
-    int units = num_sms / CG;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.blockDim = dim3(threads_of(G), 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    if (CG == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cfg.gridDim = dim3(2 * units, 1, 1);
-        int active = 0;  // clusters that fit on the device at once
-        if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 && active < units)
-            units = active;
-        (void)cudaGetLastError();
-    }
-    if (units > num_work) units = num_work;
-    cfg.gridDim = dim3(CG * units, 1, 1);
-    err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, status);
-    if (err != cudaSuccess) return err;
-    return cudaGetLastError();
 }
 
 template <int K, int G>
 cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
                       int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
                       int num_sms, cudaStream_t stream) {
-    if (cta_group() == 2)
-        return launch_kgc<K, G, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
-    return launch_kgc<K, G, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+    auto kern = router_gemm_kernel<K, G>;
+    const int stages = stages_for(Nr, K, G);
+    const size_t smem = 1024 + misc_layout(Nr, K, G, stages).total;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    const int num_work = (num_tiles + kPair - 1) / kPair;
+    int units = num_sms / kPair;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kPair;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.blockDim = dim3(threads_of(G), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.gridDim = dim3(kPair * units, 1, 1);
+    int active = 0;  // clusters that fit on the device at once
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 && active < units)
+        units = active;
+    (void)cudaGetLastError();
+    if (units > num_work) units = num_work;
+    cfg.gridDim = dim3(kPair * units, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, status);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
 }
 
 template <int K>
@@ -537,7 +487,7 @@ cudaError_t launch_k(const CUtensorMap &th, const CUtensorMap &tw, const float *
 
 }  // namespace
 
-int router_gemm_w_box_rows(int Nr) { return Nr / cta_group(); }
+int router_gemm_w_box_rows(int Nr) { return Nr / kPair; }
 
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
