@@ -217,15 +217,24 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
 
+    from expert_bias_load_b200.dp import DataParallelRouterStep, global_loads
+    rec = [None, None]  # CUDA events around the router kernel of the current step
+
+    def route(hidden, b, c):
+        if rec[0] is not None:
+            rec[0].record(stream)
+        ebl.router_forward(hidden, W, b, K, c, topk_idx=idx, gates=gates, status=status, stream=stream)
+        if rec[1] is not None:
+            rec[1].record(stream)
+
+    def update(c, b, m, mv):
+        ebl.smebu_step(c, b, m, reset_counts=True, maxvio=mv, status=status, stream=stream)
+
+    dp_step = DataParallelRouterStep(route, update)  # all-reduces the loads when world > 1
+
     def step(ev0=None, ev1=None):
-        if ev0 is not None:
-            ev0.record(stream)
-        ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=gates, status=status, stream=stream)
-        if ev1 is not None:
-            ev1.record(stream)
-        if world > 1:
-            dist.all_reduce(counts)
-        ebl.smebu_step(counts, bias, mom, reset_counts=True, maxvio=maxvio, status=status, stream=stream)
+        rec[0], rec[1] = ev0, ev1
+        dp_step(h, bias, mom, counts, maxvio)
 
     for _ in range(args.warmup):
         step()
@@ -329,8 +338,7 @@ def main():
                 ev[0].record(stream)
             ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=gates, tile_counts=tiles,
                                status=status, stream=stream)
-            if world > 1:
-                dist.all_reduce(counts)
+            global_loads(counts)
             ebl.smebu_step(counts, bias, mom, reset_counts=True, maxvio=maxvio, status=status, stream=stream)
             if rec:
                 ev[1].record(stream)

@@ -24,6 +24,7 @@ __all__ = [
     "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_logits", "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
     "read_internal_status", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD", "EBL_ST_TIMEOUT",
+    "EBL_ST_BAD_COUNTS",
     "SMEBU_LAMBDA", "SMEBU_BETA", "SMEBU_KAPPA",
 ]
 
@@ -31,7 +32,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libebl.so")
 
 EBL_OK, EBL_EINVAL, EBL_EUNSUPPORTED, EBL_ECUDA, EBL_EDATA = 0, -1, -2, -3, -4
-EBL_ST_BAD_EXPERT, EBL_ST_BAD_DEST, EBL_ST_EMPTY_LOAD, EBL_ST_TIMEOUT = 1, 2, 4, 8
+EBL_ST_BAD_EXPERT, EBL_ST_BAD_DEST, EBL_ST_EMPTY_LOAD, EBL_ST_TIMEOUT, EBL_ST_BAD_COUNTS = 1, 2, 4, 8, 16
 
 # Trinity Large's SMEBU constants ("Arcee Trinity Large Technical Report" 2.3)
 SMEBU_LAMBDA, SMEBU_BETA, SMEBU_KAPPA = 5e-4, 0.5, 2.0

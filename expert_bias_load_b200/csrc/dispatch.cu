@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(kMaxExperts) seg_sums_kernel(const int32_t *__
 }
 
 __global__ void __launch_bounds__(kMaxExperts) seg_scan_kernel(int32_t *__restrict__ seg, int num_segs, int Nr,
-                                                               int32_t *__restrict__ offsets) {
+                                                               long long num_pairs, int32_t *__restrict__ offsets,
+                                                               int32_t *__restrict__ status) {
     __shared__ int warp_tot[kMaxExperts / 32];
     const int e = threadIdx.x;
     const int lane = e & 31, warp = e >> 5;
@@ -89,7 +90,11 @@ __global__ void __launch_bounds__(kMaxExperts) seg_scan_kernel(int32_t *__restri
     const int excl = before + incl - total;
     if (e < Nr) {
         offsets[e] = excl;
-        if (e == Nr - 1) offsets[Nr] = excl + total;
+        if (e == Nr - 1) {
+            offsets[Nr] = excl + total;
+            // tile counts that do not add up to T*K cannot come from this topk_idx
+            if ((long long)excl + total != num_pairs) atomicOr(status, kStBadCounts);
+        }
         int run = excl;
         for (int s = 0; s < num_segs; ++s) {
             const int v = seg[(size_t)s * Nr + e];
@@ -261,7 +266,7 @@ cudaError_t launch_dispatch(const uint16_t *hidden, const int32_t *topk_idx, con
         tc = ws_tiles;
     }
     seg_sums_kernel<<<segs, kMaxExperts, 0, stream>>>(tc, tiles, Nr, ws_seg);
-    seg_scan_kernel<<<1, kMaxExperts, 0, stream>>>(ws_seg, segs, Nr, offsets);
+    seg_scan_kernel<<<1, kMaxExperts, 0, stream>>>(ws_seg, segs, Nr, (long long)T * K, offsets, status);
     tile_bases_kernel<<<segs, kMaxExperts, 0, stream>>>(tc, ws_seg, tiles, Nr, ws_tiles);
     int grid = num_sms * 4;
     if (grid > tiles) grid = tiles;

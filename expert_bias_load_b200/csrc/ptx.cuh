@@ -14,6 +14,7 @@ constexpr int kStBadExpert = 1;
 constexpr int kStBadDest = 2;
 constexpr int kStEmptyLoad = 4;
 constexpr int kStTimeout = 8;
+constexpr int kStBadCounts = 16;
 
 // Upper bound on any single pipeline wait inside a kernel.  Correct runs wait
 // microseconds; after this the waiting role reports EBL_ST_TIMEOUT and bails.

@@ -58,6 +58,7 @@ typedef struct CUstream_st *ebl_stream_t;
 #define EBL_ST_BAD_DEST 2     /* a dest index outside [0, T*K) was seen; that slot was skipped */
 #define EBL_ST_EMPTY_LOAD 4   /* sum of loads was 0: bias/momentum left untouched */
 #define EBL_ST_TIMEOUT 8      /* a pipeline wait inside the router kernel ran out; outputs invalid */
+#define EBL_ST_BAD_COUNTS 16  /* dispatch: tile_counts do not add up to T*K (they do not match topk_idx) */
 
 #define EBL_MAX_EXPERTS 256   /* N_r limit of every entry point */
 #define EBL_MAX_TOPK 8        /* K limit */
@@ -191,7 +192,10 @@ int sign_update_step(int32_t *counts, float *bias, int N_r, float gamma, int res
  * workspace    device scratch of at least ebl_dispatch_workspace_bytes(T, N_r)
  *              bytes, 16-byte aligned; contents on entry are ignored.
  * status       EBL_ST_BAD_EXPERT if an id is outside [0, N_r): that pair is
- *              skipped and its dest is -1.
+ *              skipped and its dest is -1.  EBL_ST_BAD_COUNTS if the given
+ *              tile_counts do not add up to T*K; destinations that would fall
+ *              outside [0, T*K) are then skipped (dest -1), others are not
+ *              meaningful.  Nothing is written outside the output buffers.
  * T*K <= 2^31 - 1.
  */
 size_t ebl_dispatch_workspace_bytes(int T, int N_r);

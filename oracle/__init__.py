@@ -55,6 +55,8 @@ def _bind(path):
     lib.orc_router_gemm.restype = i32
     lib.orc_router_logits.argtypes = [P, P, i64, i32, i32, P, P, P, P, P, i32]
     lib.orc_router_logits.restype = i32
+    lib.orc_router_zloss.argtypes = [P, P, i64, i32, i32]
+    lib.orc_router_zloss.restype = ctypes.c_double
     lib.orc_maxvio.argtypes = [P, i32, P, P]
     lib.orc_maxvio.restype = ctypes.c_double
     lib.orc_smebu.argtypes = [P, P, P, i32, f32, f32, f32, P]
@@ -174,6 +176,13 @@ def router_logits(logits, bias, K, counts=None, want_scores=False, tile_tokens=0
     if rc != ORC_OK:
         raise ValueError("orc_router_logits returned %d" % rc)
     return RouterResult(idx=idx, gates=gates, counts=cnt, scores=scores, tile_counts=tc)
+
+
+def router_zloss(hidden, W):
+    """sum_t (logsumexp_i x_{t,i})^2 of the fp64 router logits."""
+    h = _bf16_bits(hidden)
+    w = _bf16_bits(W)
+    return float(_load().orc_router_zloss(_ptr(h), _ptr(w), h.shape[0], h.shape[1], w.shape[0]))
 
 
 def maxvio(counts):

@@ -58,6 +58,14 @@ static double bf16_to_f64(uint16_t h)
     return (double)f;
 }
 
+/* sum_k a[k] * b[k * b_stride] over k < d, exact bf16 products summed in fp64. */
+static double dot_bf16(const uint16_t *a, const uint16_t *b, int64_t b_stride, int d)
+{
+    double acc = 0.0;
+    for (int k = 0; k < d; ++k) acc += bf16_to_f64(a[k]) * bf16_to_f64(b[k * b_stride]);
+    return acc;
+}
+
 /* The sigmoid router score s = 1 / (1 + exp(-x))  ([TR] 2.3; [BLOG]). */
 static double sigmoid_f64(double x)
 {
@@ -128,11 +136,8 @@ int orc_router_gemm(const uint16_t *hidden, const uint16_t *W, const float *bias
         for (int64_t t = 0; t < T; ++t) {
             const uint16_t *h = hidden + t * (int64_t)d;
             for (int i = 0; i < Nr; ++i) {
-                const uint16_t *w = W + (int64_t)i * d;
-                double acc = 0.0;
-                for (int k = 0; k < d; ++k) acc += bf16_to_f64(h[k]) * bf16_to_f64(w[k]);
-                x[i] = acc;
-                s[i] = sigmoid_f64(acc);
+                x[i] = dot_bf16(h, W + (int64_t)i * d, 1, d); /* u_t . e_i */
+                s[i] = sigmoid_f64(x[i]);
                 key[i] = s[i] + (double)bias[i];
             }
             int32_t *sel = idx + t * K;
@@ -202,6 +207,35 @@ int orc_router_logits(const float *logits, const float *bias, int64_t T, int Nr,
         for (int64_t p = 0; p < T * K; ++p) tile_counts[(p / K / tile_tokens) * Nr + idx[p]] += 1;
     }
     return ORC_OK;
+}
+
+/*
+ * Router z-loss statistic: sum over tokens of (log sum_i exp(x_{t,i}))^2, the
+ * per-token term of L_z = log^2 sum_i e^{x_i} ([TALK], "Precision Fallbacks,
+ * Loss Stabilization, and MaxVio as Data Telemetry", stabilization table;
+ * weights in [TR] section 6).  fp64; the log-sum-exp is taken around the row
+ * maximum so that large logits do not overflow.  Same inputs as
+ * orc_router_gemm.
+ */
+double orc_router_zloss(const uint16_t *hidden, const uint16_t *W, int64_t T, int d, int Nr)
+{
+    double total = 0.0;
+    double *x = (double *)malloc(sizeof(double) * (size_t)Nr);
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *h = hidden + t * (int64_t)d;
+        double mx = -INFINITY;
+        for (int i = 0; i < Nr; ++i) {
+            const double xi = dot_bf16(h, W + (int64_t)i * d, 1, d);
+            x[i] = xi;
+            if (xi > mx) mx = xi;
+        }
+        double sum = 0.0;
+        for (int i = 0; i < Nr; ++i) sum += exp(x[i] - mx);
+        const double lse = mx + log(sum);
+        total += lse * lse;
+    }
+    free(x);
+    return total;
 }
 
 /*

@@ -223,6 +223,29 @@ def pin_sigmoid_symmetry_and_rounding():
         assert np.all(np.abs(sl[mism].view(np.int32) - ref[mism].view(np.int32)) <= 1)
 
 
+# ------------------------------------------------------------- z-loss pins
+
+def pin_zloss_library_and_closed_form():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(18)
+    T, d, Nr = 50, 40, 24
+    h = _bf16(rng.standard_normal((T, d)))
+    w = _bf16(rng.standard_normal((Nr, d)) * 0.4)
+    x = _bf16_to_f64(h) @ _bf16_to_f64(w).T
+    ref = float(np.sum(logsumexp(x, axis=1) ** 2))                 # library logsumexp
+    assert abs(oracle.router_zloss(h, w) - ref) <= 1e-12 * ref
+    # all logits 0: every row is log(N_r), so the sum is T log^2 N_r
+    z = oracle.router_zloss(np.zeros((7, 8), np.uint16), w[:, :8])
+    assert abs(z - 7 * math.log(Nr) ** 2) <= 1e-12 * z
+    # shifting every logit of a row by c shifts its log-sum-exp by c (large c: no overflow)
+    hb = np.zeros((1, d), np.uint16)
+    hb[0, 0] = _bf16(np.array([64.0]))[0]
+    wb = np.zeros((Nr, d), np.uint16)
+    wb[:, 0] = _bf16(np.array([16.0]))[0]                          # every logit = 1024
+    z = oracle.router_zloss(hb, wb)
+    assert abs(z - (1024.0 + math.log(Nr)) ** 2) <= 1e-9 * z
+
+
 # -------------------------------------------------------------- SMEBU pins
 
 def pin_smebu_golden_overload():

@@ -113,3 +113,23 @@ def test_router_then_dispatch_with_router_tiles(cuda_device):
     assert np.array_equal(np.diff(o_off), to_np(counts))
     out = ebl.moe_combine(X, gates, dest)
     assert torch.allclose(out, h.float(), rtol=1e-6, atol=0)
+
+
+def test_dispatch_inconsistent_tile_counts_sets_status(cuda_device):
+    """Tile counts that do not belong to topk_idx (host-side fault injection):
+    the call reports EBL_ST_BAD_COUNTS and writes nothing out of bounds."""
+    dev = cuda_device
+    T, d, Nr, K = 1000, 64, 32, 2
+    idx = _topk_ids(T, K, Nr, seed=21).to(dev)
+    h = synth.hidden_normal(T, d, seed=22).to(dev)
+    tiles = torch.zeros(((T + 127) // 128, Nr), dtype=torch.int32, device=dev)
+    tiles[:, 0] = 500                              # far too many pairs for expert 0
+    X = torch.zeros((T * K, d), dtype=torch.bfloat16, device=dev)
+    guard = torch.full((4096,), 7, dtype=torch.int16, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    offsets, perm, dest, X = ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles, dispatched=X, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & ebl.EBL_ST_BAD_COUNTS
+    dn = to_np(dest)
+    assert np.all((dn == -1) | ((dn >= 0) & (dn < T * K)))
+    assert torch.all(guard == 7)

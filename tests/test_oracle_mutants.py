@@ -16,8 +16,8 @@ from tests import oracle_pins
 MUTANTS = {
     "sigmoid_sign": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
     "bias_on_logit": (
-        "s[i] = sigmoid_f64(acc);\n                key[i] = s[i] + (double)bias[i];",
-        "s[i] = sigmoid_f64(acc + (double)bias[i]);\n                key[i] = s[i];"),
+        "s[i] = sigmoid_f64(x[i]);\n                key[i] = s[i] + (double)bias[i];",
+        "s[i] = sigmoid_f64(x[i] + (double)bias[i]);\n                key[i] = s[i];"),
     "gates_from_keys": ("for (int k = 0; k < K; ++k) gates[t * K + k] = s[sel[k]] / sum;",
                         "for (int k = 0; k < K; ++k) gates[t * K + k] = key[sel[k]] / sum;"),
     "gates_not_normalised": ("gates[t * K + k] = s[sel[k]] / sum;", "gates[t * K + k] = s[sel[k]];"),
@@ -27,8 +27,10 @@ MUTANTS = {
                               "        taken[best] = 1;\n        out[k] = best;\n    }\n}\n\n/*\n * Router step, GEMM",
                               "            if (best < 0 || key[i] >= key[best]) best = i;\n        }\n"
                               "        taken[best] = 1;\n        out[k] = best;\n    }\n}\n\n/*\n * Router step, GEMM"),
-    "transposed_W": ("acc += bf16_to_f64(h[k]) * bf16_to_f64(w[k]);",
-                     "acc += bf16_to_f64(h[k]) * bf16_to_f64(W[(int64_t)k * Nr + i]); (void)w;"),
+    "transposed_W": ("x[i] = dot_bf16(h, W + (int64_t)i * d, 1, d);",
+                     "x[i] = dot_bf16(h, W + i, Nr, d);"),
+    "zloss_transposed_W": ("const double xi = dot_bf16(h, W + (int64_t)i * d, 1, d);",
+                           "const double xi = dot_bf16(h, W + i, Nr, d);"),
     "logits_mode_f32_sigmoid": ("s[i] = (float)sigmoid_f64((double)x[i]);",
                                 "s[i] = 1.0f / (1.0f + expf(-x[i]));"),
     "smebu_no_recentre": ("double d = db[i] - mean;", "double d = db[i];"),
@@ -46,6 +48,8 @@ MUTANTS = {
     "sign_recentre_old_b": ("for (int i = 0; i < Nr; ++i) sum += bp[i];",
                             "for (int i = 0; i < Nr; ++i) sum += (double)bias[i];"),
     "sign_of_zero": ("double sgn = (diff > 0.0) ? 1.0", "double sgn = (diff >= 0.0) ? 1.0"),
+    "zloss_not_squared": ("total += lse * lse;", "total += lse;"),
+    "zloss_no_max_shift": ("const double lse = mx + log(sum);", "const double lse = log(sum);"),
     "maxvio_inverted": ("return (double)mx / (double)mn;", "return (double)mn / (double)mx;"),
     "dispatch_unstable": ("    for (int64_t p = 0; p < P; ++p) {\n        int e = idx[p];",
                           "    for (int64_t p = P - 1; p >= 0; --p) {\n        int e = idx[p];"),
