@@ -372,6 +372,39 @@ def main():
                 "combine_frac_hbm": comb_bytes / (tc / 1e3) / 1e9 / peaks["hbm_gbs"]}
         del X, out
 
+    # ---- logits mode (the bit-exact path) and the fused z-loss on the same workload shape
+    extra = {}
+    if not args.no_full_step:
+        reps = max(3, min(20, args.steps // 50))
+        zl = torch.zeros(1, dtype=torch.float64, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for _ in range(2):
+            ebl.router_forward_zloss(h, W, bias, K, counts, zl, topk_idx=idx, gates=gates, stream=stream)
+        counts.zero_()
+        ev[0].record(stream)
+        for _ in range(reps):
+            ebl.router_forward_zloss(h, W, bias, K, counts, zl, topk_idx=idx, gates=gates, stream=stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        extra["zloss_router_ms"] = ev[0].elapsed_time(ev[1]) / reps
+        del zl
+        x = synth.logits_normal(T, Nr, seed=synth.step_seed(WORKLOAD, 1) + 1000 * rank, device=dev, quant8=True)
+        for _ in range(2):
+            ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=gates, stream=stream)
+        counts.zero_()
+        ev[0].record(stream)
+        for _ in range(reps):
+            ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=gates, stream=stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        lm = ev[0].elapsed_time(ev[1]) / reps
+        lbytes = T * Nr * 4 + T * K * 8
+        extra["logits_mode"] = {"tokens_per_s": T * world / (lm / 1e3), "ms": lm,
+                                "achieved_gbs": lbytes / (lm / 1e3) / 1e9,
+                                "frac_hbm": lbytes / (lm / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        counts.zero_()
+        del x
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, rows, threads, secs = oracle_sample(cfg, args.cpu_seconds)
@@ -388,7 +421,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-            "clocks": clk, "status": st, "maxvio_after_warmup": maxvio_first, "full_step": full}
+            "clocks": clk, "status": st, "maxvio_after_warmup": maxvio_first, "full_step": full, **extra}
     print(json.dumps(line), flush=True)
 
 

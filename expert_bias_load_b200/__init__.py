@@ -21,7 +21,7 @@ import os
 import torch
 
 __all__ = [
-    "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_logits", "smebu_step",
+    "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_logits", "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
     "read_internal_status", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD", "EBL_ST_TIMEOUT",
     "EBL_ST_BAD_COUNTS",
@@ -47,6 +47,7 @@ SIGNATURES = {
     "ebl_version": (_I, []),
     "ebl_tile_tokens": (_I, []),
     "router_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "router_forward_zloss": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "router_forward_logits": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "smebu_step": (_I, [_P, _P, _P, _I, _F, _F, _F, _I, _P, _P, _P]),
     "smebu_step_layers": (_I, [_P, _P, _P, _I, _I, _F, _F, _F, _I, _I, _P, _P, _P]),
@@ -146,6 +147,27 @@ def router_forward(hidden, W_router, bias, K, counts, topk_idx=None, gates=None,
         _check(status, "status", torch.int32, (1,))
     _call("router_forward", _ptr(hidden), _ptr(W_router), _ptr(bias), T, d, Nr, K, _ptr(topk_idx), _ptr(gates),
           _ptr(counts), _ptr(tile_counts), _ptr(status), _stream(stream))
+    return topk_idx, gates
+
+
+def router_forward_zloss(hidden, W_router, bias, K, counts, zloss_sum, topk_idx=None, gates=None, tile_counts=None,
+                         status=None, stream=None):
+    """router_forward that also adds sum_t logsumexp(x_t)^2 into zloss_sum
+    (fp64 [1], caller-zeroed).  Returns (topk_idx, gates)."""
+    _check(hidden, "hidden", torch.bfloat16)
+    T, d = hidden.shape
+    Nr = W_router.shape[0]
+    _check(W_router, "W_router", torch.bfloat16, (Nr, d))
+    _check(bias, "bias", torch.float32, (Nr,))
+    _check(counts, "counts", torch.int32, (Nr,))
+    _check(zloss_sum, "zloss_sum", torch.float64, (1,))
+    dev = hidden.device
+    topk_idx = _out(topk_idx, "topk_idx", (T, K), torch.int32, dev)
+    gates = _out(gates, "gates", (T, K), torch.float32, dev)
+    if tile_counts is not None:
+        _check(tile_counts, "tile_counts", torch.int32, ((T + 127) // 128, Nr))
+    _call("router_forward_zloss", _ptr(hidden), _ptr(W_router), _ptr(bias), T, d, Nr, K, _ptr(topk_idx),
+          _ptr(gates), _ptr(counts), _ptr(tile_counts), _ptr(zloss_sum), _ptr(status), _stream(stream))
     return topk_idx, gates
 
 

@@ -92,6 +92,36 @@ int check_T(int T) { return (T < 0 || T > 2147483647 - 255) ? EBL_EINVAL : EBL_O
 
 }  // namespace
 
+namespace {
+
+int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d, int N_r,
+                     int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                     double *zloss_sum, int32_t *status, ebl_stream_t stream) {
+    if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
+    if (d < 64 || d > (1 << 20) || d % 64 != 0) return EBL_EINVAL;
+    if (N_r % 32 != 0) return EBL_EUNSUPPORTED;
+    if (!hidden || !W_router || !bias || !topk_idx || !gates || !counts) return EBL_EINVAL;
+    if (!aligned16(hidden) || !aligned16(W_router) || !aligned4(bias) || !aligned4(counts)) return EBL_EINVAL;
+    if (K % 4 == 0 && (!aligned16(topk_idx) || !aligned16(gates))) return EBL_EINVAL;
+    if (!aligned4(topk_idx) || !aligned4(gates) || (tile_counts && !aligned4(tile_counts))) return EBL_EINVAL;
+    if (zloss_sum && (reinterpret_cast<uintptr_t>(zloss_sum) & 7u)) return EBL_EINVAL;
+    if (T == 0) return EBL_OK;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    if ((rc = get_encoder())) return rc;
+    CUtensorMap th, tw;
+    if ((rc = encode_bf16_2d(&th, hidden, (uint64_t)T, (uint64_t)d, ebl::kTileTokens))) return rc;
+    if ((rc = encode_bf16_2d(&tw, W_router, (uint64_t)N_r, (uint64_t)d, (uint32_t)ebl::router_gemm_w_box_rows(N_r))))
+        return rc;
+    cudaError_t e = ebl::launch_router_gemm(th, tw, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts,
+                                            zloss_sum, status ? status : di.internal_status, di.num_sms,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EBL_OK : cuda_fail();
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *ebl_strerror(int code) {
@@ -118,26 +148,16 @@ int ebl_tile_tokens(void) { return ebl::kTileTokens; }
 int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d, int N_r,
                    int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
                    ebl_stream_t stream) {
-    if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
-    if (d < 64 || d > (1 << 20) || d % 64 != 0) return EBL_EINVAL;
-    if (N_r % 32 != 0) return EBL_EUNSUPPORTED;
-    if (!hidden || !W_router || !bias || !topk_idx || !gates || !counts) return EBL_EINVAL;
-    if (!aligned16(hidden) || !aligned16(W_router) || !aligned4(bias) || !aligned4(counts)) return EBL_EINVAL;
-    if (K % 4 == 0 && (!aligned16(topk_idx) || !aligned16(gates))) return EBL_EINVAL;
-    if (!aligned4(topk_idx) || !aligned4(gates) || (tile_counts && !aligned4(tile_counts))) return EBL_EINVAL;
-    if (T == 0) return EBL_OK;
-    DeviceInfo di;
-    int rc = device_info(&di);
-    if (rc) return rc;
-    if ((rc = get_encoder())) return rc;
-    CUtensorMap th, tw;
-    if ((rc = encode_bf16_2d(&th, hidden, (uint64_t)T, (uint64_t)d, ebl::kTileTokens))) return rc;
-    if ((rc = encode_bf16_2d(&tw, W_router, (uint64_t)N_r, (uint64_t)d, (uint32_t)ebl::router_gemm_w_box_rows(N_r))))
-        return rc;
-    cudaError_t e = ebl::launch_router_gemm(th, tw, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts,
-                                            status ? status : di.internal_status, di.num_sms,
-                                            reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return router_gemm_call(hidden, W_router, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts, nullptr,
+                            status, stream);
+}
+
+int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d,
+                         int N_r, int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                         double *zloss_sum, int32_t *status, ebl_stream_t stream) {
+    if (!zloss_sum) return EBL_EINVAL;
+    return router_gemm_call(hidden, W_router, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts, zloss_sum,
+                            status, stream);
 }
 
 int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K, int32_t *topk_idx,

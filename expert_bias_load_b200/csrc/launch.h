@@ -18,7 +18,8 @@ constexpr int kMaxTopK = 8;       // K limit
 int router_gemm_w_box_rows(int Nr);  // rows of W per TMA box (N_r / CTAs per MMA)
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
-                               int32_t *tile_counts, int32_t *status, int num_sms, cudaStream_t stream);
+                               int32_t *tile_counts, double *zloss_sum, int32_t *status, int num_sms,
+                               cudaStream_t stream);
 
 // router_logits.cu
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,

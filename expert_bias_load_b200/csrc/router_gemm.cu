@@ -75,7 +75,8 @@ __host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int stages) {
     // full[S], empty[S], tfull[2], tempty[2], epi_sync, drain, list_full, list_empty; tmem slot, abort flag
     const size_t bars = (size_t)(2 * stages + 8) * 8 + 16;
     m.vec_off = m.bar_off + ((bars + 15) & ~size_t(15));
-    const size_t vec = (size_t)4 * Nr * 4 + (size_t)3 * (G - 1) * K * kTileTokens * 4;
+    const size_t vec = (size_t)4 * Nr * 4 + (size_t)3 * (G - 1) * K * kTileTokens * 4 +
+                       (size_t)2 * (G - 1) * kTileTokens * 4;  // partial lists; partial log-sum-exp
     m.total = m.vec_off + vec;
     return m;
 }
@@ -87,9 +88,32 @@ __device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-template <int K>
+// Running log-sum-exp of a row's logits as (max, sum of exp(x - max)).
+struct RowLse {
+    float m, s;
+    __device__ __forceinline__ void init() {
+        m = -INFINITY;
+        s = 0.0f;
+    }
+    __device__ __forceinline__ void merge(float m2, float s2) {
+        const float nm = fmaxf(m, m2);
+        s = s * __expf(m - nm) + s2 * __expf(m2 - nm);
+        m = nm;
+    }
+};
+
+template <int K, bool Z>
 __device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const float *__restrict__ bias_s, int c,
-                                              RowTopK<K> &tk) {
+                                              RowTopK<K> &tk, RowLse &lse) {
+    if constexpr (Z) {  // z-loss: log-sum-exp of the chunk, folded into the row's
+        float cm = __uint_as_float(r[0]);
+#pragma unroll
+        for (int j = 1; j < kChunk; ++j) cm = fmaxf(cm, __uint_as_float(r[j]));
+        float cs = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) cs += __expf(__uint_as_float(r[j]) - cm);
+        lse.merge(cm, cs);
+    }
     const float4 *b4 = reinterpret_cast<const float4 *>(bias_s + c);
 #pragma unroll
     for (int q = 0; q < kChunk / 4; ++q) {
@@ -104,12 +128,13 @@ __device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const
     }
 }
 
-template <int K, int G>
+template <int K, int G, bool Z>
 __global__ void __launch_bounds__(threads_of(G), 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
                        const float *__restrict__ bias, int T, int d, int Nr, int stages,
                        int32_t *__restrict__ topk_idx, float *__restrict__ gates, int32_t *__restrict__ counts,
-                       int32_t *__restrict__ tile_counts, int32_t *__restrict__ status) {
+                       int32_t *__restrict__ tile_counts, double *__restrict__ zloss_sum,
+                       int32_t *__restrict__ status) {
     constexpr int kEpiWarps = 4 * G;
     constexpr int kProducerWarp = 4 * G;
     constexpr int kMmaWarp = 4 * G + 1;
@@ -136,6 +161,8 @@ __global__ void __launch_bounds__(threads_of(G), 1)
     float *pl_key = reinterpret_cast<float *>(hist_tile + 2 * Nr);  // [G-1][K][128]
     float *pl_s = pl_key + (G - 1) * K * kTileTokens;
     int *pl_idx = reinterpret_cast<int *>(pl_s + (G - 1) * K * kTileTokens);
+    float *pl_zm = reinterpret_cast<float *>(pl_idx + (G - 1) * K * kTileTokens);  // [G-1][128]
+    float *pl_zs = pl_zm + (G - 1) * kTileTokens;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -286,6 +313,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         uint32_t sync_ph = 0;
         bool ok = true;
         int it = 0;
+        float zacc = 0.0f;  // this thread's rows: sum of log-sum-exp squared
         for (int wk = unit; wk < num_work; wk += num_units, ++it) {
             const int tile = wk * kPair + (int)rank;
             const int acc = it & 1;
@@ -298,6 +326,8 @@ __global__ void __launch_bounds__(threads_of(G), 1)
 
             RowTopK<K> tk;
             tk.init();
+            RowLse lse;
+            lse.init();
             const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * Nr + c0);
             uint32_t ra[kChunk], rb[kChunk];
             __syncwarp();
@@ -306,12 +336,12 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             for (int c = 0; c < cpg; c += 2 * kChunk) {  // cpg % 32 == 0: chunks come in pairs
                 __syncwarp();
                 tmem_ld_32x32b_x16(taddr + (uint32_t)(c + kChunk), rb);
-                consume_chunk<K>(ra, bias_s, c0 + c, tk);
+                consume_chunk<K, Z>(ra, bias_s, c0 + c, tk, lse);
                 __syncwarp();
                 tmem_ld_wait_x16(rb);
                 const bool more = c + 2 * kChunk < cpg;
                 if (more) tmem_ld_32x32b_x16(taddr + (uint32_t)(c + 2 * kChunk), ra);
-                consume_chunk<K>(rb, bias_s, c0 + c + kChunk, tk);
+                consume_chunk<K, Z>(rb, bias_s, c0 + c + kChunk, tk, lse);
                 __syncwarp();
                 if (more) tmem_ld_wait_x16(ra);
             }
@@ -333,6 +363,10 @@ __global__ void __launch_bounds__(threads_of(G), 1)
                     pl_s[base + k * kTileTokens] = tk.score[k];
                     pl_idx[base + k * kTileTokens] = tk.idx[k];
                 }
+                if constexpr (Z) {
+                    pl_zm[(group - 1) * kTileTokens + rloc] = lse.m;
+                    pl_zs[(group - 1) * kTileTokens + rloc] = lse.s;
+                }
                 mbar_arrive(list_full);
                 continue;
             }
@@ -353,12 +387,19 @@ __global__ void __launch_bounds__(threads_of(G), 1)
                         if (!(kv > tk.key[K - 1])) break;
                         tk.push(kv, pl_s[base + k * kTileTokens], pl_idx[base + k * kTileTokens]);
                     }
+                    if constexpr (Z) lse.merge(pl_zm[(g - 1) * kTileTokens + rloc], pl_zs[(g - 1) * kTileTokens + rloc]);
                 }
                 mbar_arrive(list_empty);
             }
 
             const int row = tile * kTileTokens + rloc;
             int *hist = want_tiles ? hist_tile + (it & 1) * Nr : hist_total;
+            if constexpr (Z) {
+                if (row < T) {
+                    const float l = lse.m + logf(lse.s);
+                    zacc += l * l;
+                }
+            }
             if (row < T) {
                 float sum = 0.0f;
 #pragma unroll
@@ -410,6 +451,12 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             if (ok) {
                 for (int e = rloc; e < Nr; e += 128)
                     if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
+                if constexpr (Z) {  // one fp64 atomic per warp
+                    double z = (double)zacc;
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+                    if (lane == 0) atomicAdd(zloss_sum, z);
+                }
             }
         }
         if (!ok) {
@@ -429,7 +476,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
 
 int groups_for(int Nr) { return (Nr % 128 == 0) ? 4 : ((Nr % 64 == 0) ? 2 : 1); }
 
-int stages_for(int Nr, int K, int G) {
+int stages_for(int Nr, int K, int G) {  // the layout is the same with and without z-loss
     const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
     int s = kMaxStages;
     while (s > 2 && 1024 + misc_layout(Nr, K, G, s).total > budget) --s;
@@ -438,9 +485,9 @@ int stages_for(int Nr, int K, int G) {
 
 template <int K, int G>
 cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
-                      int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
-                      int num_sms, cudaStream_t stream) {
-    auto kern = router_gemm_kernel<K, G>;
+                      int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zloss_sum,
+                      int32_t *status, int num_sms, cudaStream_t stream) {
+    auto kern = zloss_sum ? router_gemm_kernel<K, G, true> : router_gemm_kernel<K, G, false>;
     const int stages = stages_for(Nr, K, G);
     const size_t smem = 1024 + misc_layout(Nr, K, G, stages).total;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -466,22 +513,23 @@ cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float 
     (void)cudaGetLastError();
     if (units > num_work) units = num_work;
     cfg.gridDim = dim3(kPair * units, 1, 1);
-    err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, status);
+    err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, zloss_sum,
+                             status);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 template <int K>
 cudaError_t launch_k(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
-                     int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
-                     int num_sms, cudaStream_t stream) {
+                     int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zl,
+                     int32_t *status, int num_sms, cudaStream_t stream) {
     switch (groups_for(Nr)) {
         case 4:
-            return launch_kg<K, 4>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+            return launch_kg<K, 4>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
         case 2:
-            return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+            return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
         default:
-            return launch_kg<K, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, status, num_sms, stream);
+            return launch_kg<K, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
     }
 }
 
@@ -491,11 +539,13 @@ int router_gemm_w_box_rows(int Nr) { return Nr / kPair; }
 
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
-                               int32_t *tile_counts, int32_t *status, int num_sms, cudaStream_t stream) {
+                               int32_t *tile_counts, double *zloss_sum, int32_t *status, int num_sms,
+                               cudaStream_t stream) {
     switch (K) {
 #define EBL_CASE(KK) \
     case KK:         \
-        return launch_k<KK>(tmap_h, tmap_w, bias, T, d, Nr, topk_idx, gates, counts, tile_counts, status, num_sms, stream);
+        return launch_k<KK>(tmap_h, tmap_w, bias, T, d, Nr, topk_idx, gates, counts, tile_counts, zloss_sum, status, \
+                             num_sms, stream);
         EBL_CASE(1)
         EBL_CASE(2)
         EBL_CASE(3)

@@ -8,12 +8,22 @@
 // Sources: "Arcee Trinity Large Technical Report" section 2.3; "SMEBU Load
 // Balancing" eq. (17).
 //
-// Layout: one warp per token row; lane l owns experts l, l+32, ... (so each
-// load instruction reads 128 contiguous bytes of the row), keeps a running
-// Top-K of its own experts, and the warp merges the 32 lists with K rounds of
-// a shuffle arg-max under the order (key desc, index asc).  One CTA of 8 warps
-// handles a 128-token tile at a time (persistent grid), with a shared-memory
-// histogram flushed per tile (tile_counts) and per CTA (counts).
+// Layout: one thread per token row (a CTA of 128 threads takes a 128-token
+// tile; persistent grid).  Each thread streams its row with 16-byte loads (the
+// warp's 32 rows share L1 lines, so every fetched line is used in full) and
+// keeps a running Top-K in registers, visiting experts in increasing index so
+// that a strict comparison keeps the lower index first on equal keys.  A
+// shared-memory histogram is flushed per tile (tile_counts) and per CTA
+// (counts).
+//
+// The fp64 sigmoid is only evaluated where it can matter.  A first pass ranks
+// the experts with an fp32 sigmoid whose distance to the fp64-rounded value
+// is bounded (kSigmaErr); its K-th key tau bounds the exact K-th key within
+// kSigmaErr plus the rounding of the key add.  Only experts whose approximate
+// key is within twice that margin of tau can be in the exact Top-K, so the
+// second pass computes the exact score of those candidates alone (usually K or
+// K+1 of them) and selects among them: the same result as evaluating every
+// expert in fp64.
 
 #include "launch.h"
 #include "ptx.cuh"
@@ -22,13 +32,37 @@
 namespace ebl {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kThreads = kTileTokens;  // one thread per row of a tile
 
 __device__ __forceinline__ float sigmoid_rounded_once(float x) {
     // fp64 evaluation, one rounding to fp32 at the end
     const double e = exp(-(double)x);
     return __double2float_rn(__ddiv_rn(1.0, __dadd_rn(1.0, e)));
+}
+
+// fp32 sigmoid from the fast intrinsics: __expf (at most 2 + 1.173|x| ulp off)
+// and __fdividef (at most 2 ulp).  Its distance to sigmoid_rounded_once() is
+// below 4e-7 for every finite x (the exp error is damped by s(1-s), which
+// decays faster than the error grows); kSigmaErr leaves a 10x margin.
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+constexpr float kSigmaErr = 4.0e-6f;
+
+// Visit the row's experts in increasing index, 4 at a time when the row is
+// 16-byte aligned; f(c, x) is called for each expert c with its logit x.
+template <class F>
+__device__ __forceinline__ void for_each_logit(const float *__restrict__ x, int Nr, bool vec4, F &&f) {
+    if (vec4) {
+        const float4 *x4 = reinterpret_cast<const float4 *>(x);
+        for (int c = 0; c < Nr; c += 4) {
+            const float4 v = __ldg(x4 + (c >> 2));
+            f(c, v.x);
+            f(c + 1, v.y);
+            f(c + 2, v.z);
+            f(c + 3, v.w);
+        }
+    } else {
+        for (int c = 0; c < Nr; ++c) f(c, __ldg(x + c));
+    }
 }
 
 template <int K>
@@ -42,8 +76,6 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < Nr; i += kThreads) {
         bias_s[i] = bias[i];
         hist_total[i] = 0;
@@ -52,64 +84,42 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
     __syncthreads();
 
     const bool want_tiles = tile_counts != nullptr;
+    const bool vec4 = (Nr & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
     int *hist = want_tiles ? hist_tile : hist_total;
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
 
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        for (int r = warp; r < kTileTokens; r += kWarps) {
-            const int row = tile * kTileTokens + r;
-            if (row >= T) break;
+        const int row = tile * kTileTokens + threadIdx.x;
+        if (row < T) {
             const float *x = logits + (size_t)row * Nr;
-
-            RowTopK<K> mine;
-            mine.init();
-            for (int c = lane; c < Nr; c += 32) {
-                const float s = sigmoid_rounded_once(__ldcs(x + c));
-                mine.push(__fadd_rn(s, bias_s[c]), s, c);
-            }
-
-            int sel_i[K];
-            float sel_s[K];
+            // pass 1: approximate keys, their K-th largest
+            RowTopK<K> approx;
+            approx.init();
+            for_each_logit(x, Nr, vec4, [&](int c, float xv) {
+                approx.push(__fadd_rn(sigmoid_fast(xv), bias_s[c]), 0.0f, c);
+            });
+            const float tau = approx.key[K - 1];
+            // |approximate key - exact key| <= kSigmaErr + one rounding of each add
+            const float lim = tau - 2.0f * (kSigmaErr + 2.384185791015625e-7f * fabsf(tau));
+            // pass 2: exact keys of the candidates only
+            RowTopK<K> tk;
+            tk.init();
+            for_each_logit(x, Nr, vec4, [&](int c, float xv) {
+                if (__fadd_rn(sigmoid_fast(xv), bias_s[c]) >= lim) {
+                    const float s = sigmoid_rounded_once(xv);
+                    tk.push(__fadd_rn(s, bias_s[c]), s, c);
+                }
+            });
+            double sum = 0.0;
+#pragma unroll
+            for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)tk.score[k]);
+            int32_t *oi = topk_idx + (size_t)row * K;
+            float *og = gates + (size_t)row * K;
 #pragma unroll
             for (int k = 0; k < K; ++k) {
-                float bk = mine.key[0];
-                int bi = mine.idx[0];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) {
-                    const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                    if (ok > bk || (ok == bk && oi < bi)) {
-                        bk = ok;
-                        bi = oi;
-                    }
-                }
-                const int owner = bi & 31;
-                sel_i[k] = bi;
-                sel_s[k] = __shfl_sync(0xffffffffu, mine.score[0], owner);
-                if (lane == owner) {  // pop the head of the owner's list
-#pragma unroll
-                    for (int p = 0; p + 1 < K; ++p) {
-                        mine.key[p] = mine.key[p + 1];
-                        mine.score[p] = mine.score[p + 1];
-                        mine.idx[p] = mine.idx[p + 1];
-                    }
-                    mine.key[K - 1] = -INFINITY;
-                    mine.idx[K - 1] = 0x7fffffff;
-                }
-            }
-
-            if (lane == 0) {
-                double sum = 0.0;
-#pragma unroll
-                for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)sel_s[k]);
-                int32_t *oi = topk_idx + (size_t)row * K;
-                float *og = gates + (size_t)row * K;
-#pragma unroll
-                for (int k = 0; k < K; ++k) {
-                    oi[k] = sel_i[k];
-                    og[k] = __double2float_rn(__ddiv_rn((double)sel_s[k], sum));
-                    if ((unsigned)sel_i[k] < (unsigned)Nr) atomicAdd(&hist[sel_i[k]], 1);
-                }
+                oi[k] = tk.idx[k];
+                og[k] = __double2float_rn(__ddiv_rn((double)tk.score[k], sum));
+                if ((unsigned)tk.idx[k] < (unsigned)Nr) atomicAdd(&hist[tk.idx[k]], 1);
             }
         }
         if (want_tiles) {
@@ -134,7 +144,7 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
                                  float *gates, int32_t *counts, int32_t *tile_counts, int num_sms,
                                  cudaStream_t stream) {
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
-    int grid = num_sms * 8;
+    int grid = num_sms * 16;
     if (grid > num_tiles) grid = num_tiles;
     switch (K) {
 #define EBL_CASE(KK)                                                                                    \

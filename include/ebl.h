@@ -110,6 +110,24 @@ int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float
                    int32_t *status, ebl_stream_t stream);
 
 /*
+ * router_forward_zloss -- router_forward that also accumulates the router
+ * z-loss statistic  zloss_sum += sum_{t<T} (log sum_i exp(x_{t,i}))^2  into a
+ * caller-zeroed fp64 device scalar (one atomic per epilogue warp per CTA).
+ * The z-loss, L_z = log^2 sum_i e^{x_i} per token, is named in "Arcee Halts
+ * 400B Blackwell Model Collapse With Dynamic Router Biases" ("Precision
+ * Fallbacks, Loss Stabilization, and MaxVio as Data Telemetry", stabilization
+ * table); "Arcee Trinity Large Technical Report" section 6 gives its weight
+ * (1e-4 intended, 1e-6 effective).  The mean z-loss is zloss_sum / T.  The
+ * log-sum-exp is formed from the fp32 logits around the row maximum (no
+ * overflow).  zloss_sum: device, 8-byte aligned, not NULL.  Other arguments
+ * and outputs as router_forward.
+ */
+int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const float *bias,
+                         int T, int d, int N_r, int K,
+                         int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                         double *zloss_sum, int32_t *status, ebl_stream_t stream);
+
+/*
  * router_forward_logits -- the same selection, gates and counts from
  * precomputed fp32 logits.  This is the bit-exact mode: each value that
  * decides a selection has one defined rounding,

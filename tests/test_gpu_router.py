@@ -141,3 +141,30 @@ def test_gemm_mode_tiny_workload_smebu_steps(cuda_device):
         assert rel_err(to_np(m_g), m_o).max() <= STATE_RTOL
         assert float(maxvio.item()) == np.float32(oracle.maxvio(n_gpu)[0])
         assert int(counts.sum().item()) == 0
+
+
+ZLOSS_CASES = [(2048 + 77, 256, 64, 4), (3000, 512, 256, 4), (1000, 2048, 128, 8), (129, 64, 96, 3)]
+
+
+@pytest.mark.parametrize("T,d,Nr,K", ZLOSS_CASES)
+def test_router_zloss_vs_oracle(cuda_device, T, d, Nr, K):
+    """Fused z-loss statistic: sum_t logsumexp(x_t)^2 within 1e-4 relative of the
+    fp64 oracle (fp32 logits and exp/log: per-token error ~1e-5 relative), and
+    the routing outputs bit-identical to router_forward."""
+    dev = cuda_device
+    h = synth.hidden_normal(T, d, seed=T + 3 * d, device=dev)
+    W = synth.router_weight(Nr, d, seed=Nr + d).to(dev)
+    bias = (torch.randn(Nr, generator=torch.Generator().manual_seed(5)) * 0.02).to(dev)
+    c1 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    c2 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    z = torch.zeros(1, dtype=torch.float64, device=dev)
+    i1, g1 = ebl.router_forward(h, W, bias, K, c1)
+    i2, g2 = ebl.router_forward_zloss(h, W, bias, K, c2, z)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, i2) and torch.equal(g1, g2) and torch.equal(c1, c2)
+    ref = oracle.router_zloss(h.cpu(), W.cpu())
+    assert abs(float(z.item()) - ref) <= 1e-4 * ref, (float(z.item()), ref)
+    # accumulates: a second call adds the same amount again
+    ebl.router_forward_zloss(h, W, bias, K, c2, z)
+    torch.cuda.synchronize()
+    assert abs(float(z.item()) - 2 * ref) <= 2e-4 * ref
