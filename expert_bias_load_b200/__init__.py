@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_dispatch_static": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "ebl_read_internal_status": (_I, [_P, _I]),
+    "ebl_selftest_wait_timeout": (_I, [_P, ctypes.c_uint, _P]),
 }
 
 
@@ -269,3 +270,9 @@ def read_internal_status(clear=True) -> int:
     v = ctypes.c_int32(0)
     _call("ebl_read_internal_status", ctypes.c_void_p(ctypes.addressof(v)), int(bool(clear)))
     return int(v.value)
+
+
+def selftest_wait_timeout(status, limit_us=20000, stream=None):
+    """Run the bounded-wait self-test; EBL_ST_TIMEOUT lands in status (int32 [1])."""
+    _check(status, "status", torch.int32, (1,))
+    _call("ebl_selftest_wait_timeout", _ptr(status), int(limit_us), _stream(stream))

@@ -21,7 +21,7 @@
 //               K=16, 8 per stage) for the pair into a double-buffered
 //               fp32 accumulator (2 x N_r columns per CTA), so the epilogue of
 //               tile i overlaps the MMAs of tile i+1.
-//   epilogue    G groups of 4 warps.  Warp w reads TMEM lane quadrant w%4 (one
+//   epilogue    G = 2 (or 1) groups of 4 warps.  Warp w reads TMEM lane quadrant w%4 (one
 //               token row per thread); group g = w/4 owns the experts
 //               [g*N_r/G, (g+1)*N_r/G).  Each thread runs sigmoid, +bias and a
 //               running Top-K over its experts; groups 1..G-1 hand their
@@ -474,7 +474,10 @@ __global__ void __launch_bounds__(threads_of(G), 1)
     }
 }
 
-int groups_for(int Nr) { return (Nr % 128 == 0) ? 4 : ((Nr % 64 == 0) ? 2 : 1); }
+// Epilogue groups: 2 (8 warps, 2 per SM sub-partition) whenever the experts split
+// into 32-column halves.  Measured on the tie workload, 8 epilogue warps keep up
+// with the MMAs and leave more issue slots to the TMA and MMA warps than 16.
+int groups_for(int Nr) { return (Nr % 64 == 0) ? 2 : 1; }
 
 int stages_for(int Nr, int K, int G) {  // the layout is the same with and without z-loss
     const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
@@ -524,8 +527,6 @@ cudaError_t launch_k(const CUtensorMap &th, const CUtensorMap &tw, const float *
                      int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zl,
                      int32_t *status, int num_sms, cudaStream_t stream) {
     switch (groups_for(Nr)) {
-        case 4:
-            return launch_kg<K, 4>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
         case 2:
             return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
         default:

@@ -1,0 +1,34 @@
+// selftest.cu -- checks the bounded pipeline wait that every kernel here uses:
+// one thread waits, with a short limit, on an mbarrier that nothing arrives
+// on.  The wait must give up, the kernel must report EBL_ST_TIMEOUT in the
+// status word and return, and the CUDA context must stay usable.
+
+#include "../../include/ebl.h"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace ebl {
+namespace {
+
+__global__ void wait_timeout_kernel(int32_t *__restrict__ status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);  // expects one arrival that never comes
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicOr(status, kStTimeout);
+}
+
+}  // namespace
+}  // namespace ebl
+
+extern "C" int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us, ebl_stream_t stream) {
+    if (!status || (reinterpret_cast<uintptr_t>(status) & 3u)) return EBL_EINVAL;
+    if (limit_us < 1 || limit_us > 1000000) return EBL_EINVAL;
+    ebl::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status, 1000ull * limit_us);
+    if (cudaGetLastError() != cudaSuccess) return EBL_ECUDA;
+    return EBL_OK;
+}

@@ -272,6 +272,17 @@ int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *d
                 int T, int d, int K, float *out, int32_t *status, ebl_stream_t stream);
 
 /*
+ * ebl_selftest_wait_timeout -- failure-detection self-test.  Launches one
+ * thread that waits, through the same bounded mbarrier wait the router kernel
+ * uses for its pipeline, on a barrier nothing ever arrives on.  After
+ * limit_us microseconds (1 .. 1e6) the wait gives up and EBL_ST_TIMEOUT is
+ * OR-ed into *status (device int32); the kernel then returns and the CUDA
+ * context stays usable.  No counterpart on the pages: it exists so that the
+ * timeout path is exercised without faulting or hanging a GPU.
+ */
+int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us, ebl_stream_t stream);
+
+/*
  * ebl_read_internal_status -- copy the library-owned status word (used when a
  * call passed status == NULL) of the current device to *out, and clear it if
  * `clear` is nonzero.  Synchronous (waits for the device).
