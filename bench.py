@@ -129,32 +129,44 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle leg
 
-def oracle_sample(cfg, seconds, seed=0):
-    """Time the CPU oracle (router in fp64 + SMEBU) on a bounded sample of the
-    workload's rows; returns (tokens_per_s, rows, threads, seconds)."""
-    import numpy as np
-    import oracle
-    import synth
-    T, d, Nr, K = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"]
-    oracle.build()
-    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d)
-    bias = synth.dead_start_bias(Nr).numpy()
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+class OracleSample:
+    """The CPU oracle (fp64 router GEMM + Top-K + gates + counts, then SMEBU)
+    on a bounded sample of the workload's rows."""
 
-    def run(rows):
-        h = synth.hidden_normal(rows, d, seed=seed + rows, quant8=True)
-        b = bias.copy()
-        m = np.zeros(Nr, np.float32)
+    def __init__(self, cfg):
+        import numpy as np
+        import oracle
+        import synth
+        self.np, self.oracle, self.synth = np, oracle, synth
+        self.cfg = cfg
+        oracle.build()
+        d, Nr = cfg["d"], cfg["Nr"]
+        self.W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d)
+        self.bias = synth.dead_start_bias(Nr).numpy()
+        self.threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+    def run(self, rows, seed):
+        """Seconds the oracle takes for `rows` tokens (inputs made outside the timing)."""
+        h = self.synth.hidden_normal(rows, self.cfg["d"], seed=seed, quant8=True)
+        b = self.bias.copy()
+        m = self.np.zeros(self.cfg["Nr"], self.np.float32)
         t0 = time.perf_counter()
-        r = oracle.router_gemm(h, W, b, K)
-        oracle.smebu(r.counts, b, m)
+        r = self.oracle.router_gemm(h, self.W, b, self.cfg["K"])
+        self.oracle.smebu(r.counts, b, m)
         return time.perf_counter() - t0
 
-    rows = 64
-    t = run(rows)
-    rows = int(max(64, min(T, rows * seconds / max(t, 1e-3))))
-    t = run(rows)
-    return rows / t, rows, threads, t
+    def rows_for(self, seconds):
+        t = self.run(64, seed=1)
+        return int(max(16, min(self.cfg["T"], 64 * seconds / max(t, 1e-4))))
+
+
+def oracle_sample(cfg, seconds, seed=0):
+    """Time the oracle on a sample sized for about `seconds` of CPU work;
+    returns (tokens_per_s, rows, threads, seconds)."""
+    o = OracleSample(cfg)
+    rows = o.rows_for(seconds)
+    t = o.run(rows, seed)
+    return rows / t, rows, o.threads, t
 
 
 # ------------------------------------------------------------------- GPU leg
@@ -178,12 +190,17 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        # each step routes a bounded sample of the workload on the host cores,
+        # sized so that the whole run takes about two minutes
+        o = OracleSample(cfg)
+        per_step = min(3.0, max(0.05, 120.0 / (args.warmup + args.steps)))
+        rows = o.rows_for(per_step)
+        threads = o.threads
         vals = []
-        rows = threads = None
         for s in range(args.warmup + args.steps):
-            v, rows, threads, secs = oracle_sample(cfg, max(1.0, args.cpu_seconds / 4), seed=s)
+            t = o.run(rows, seed=s)
             if s >= args.warmup:
-                vals.append(v)
+                vals.append(rows / t)
         v = statistics.median(vals)
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": rows / v * 1e3,
