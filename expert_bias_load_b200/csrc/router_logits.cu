@@ -9,12 +9,13 @@
 // Balancing" eq. (17).
 //
 // Layout: one thread per token row (a CTA of 128 threads takes a 128-token
-// tile; persistent grid).  Each thread streams its row with 16-byte loads (the
-// warp's 32 rows share L1 lines, so every fetched line is used in full) and
-// keeps a running Top-K in registers, visiting experts in increasing index so
-// that a strict comparison keeps the lower index first on equal keys.  A
-// shared-memory histogram is flushed per tile (tile_counts) and per CTA
-// (counts).
+// tile; persistent grid).  A warp's 32 rows are read together, 32 experts at a
+// time: each load instruction fetches 128 contiguous bytes of one row, and the
+// 32 x 32 block is transposed through padded shared memory so that every thread
+// then walks its own row in increasing expert index.  Each thread keeps a
+// running Top-K in registers; visiting experts in increasing index lets a
+// strict comparison keep the lower index first on equal keys.  A shared-memory
+// histogram is flushed per tile (tile_counts) and per CTA (counts).
 //
 // The fp64 sigmoid is only evaluated where it can matter.  A first pass ranks
 // the experts with an fp32 sigmoid whose distance to the fp64-rounded value
@@ -47,21 +48,44 @@ __device__ __forceinline__ float sigmoid_rounded_once(float x) {
 __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 constexpr float kSigmaErr = 4.0e-6f;
 
-// Visit the row's experts in increasing index, 4 at a time when the row is
-// 16-byte aligned; f(c, x) is called for each expert c with its logit x.
-template <class F>
-__device__ __forceinline__ void for_each_logit(const float *__restrict__ x, int Nr, bool vec4, F &&f) {
-    if (vec4) {
-        const float4 *x4 = reinterpret_cast<const float4 *>(x);
-        for (int c = 0; c < Nr; c += 4) {
-            const float4 v = __ldg(x4 + (c >> 2));
-            f(c, v.x);
-            f(c + 1, v.y);
-            f(c + 2, v.z);
-            f(c + 3, v.w);
+constexpr int kWarpsPerCta = kThreads / 32;
+
+// The K largest values seen so far (with repeats), sorted descending; one
+// fmax/fmin pair per slot and value, no branches.  NaN values are dropped.
+template <int K>
+struct TopValues {
+    float v[K];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int k = 0; k < K; ++k) v[k] = -INFINITY;
+    }
+    __device__ __forceinline__ void push(float x) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            const float hi = fmaxf(v[k], x);
+            x = fminf(v[k], x);
+            v[k] = hi;
         }
-    } else {
-        for (int c = 0; c < Nr; ++c) f(c, __ldg(x + c));
+    }
+};
+
+// The warp's rows row0 .. row0+31 (lane l owns row0 + l): calls f(c, x) for
+// each expert c of the lane's row in increasing c, x its logit.  Rows at or
+// past T read nothing (x = 0).
+template <class F>
+__device__ __forceinline__ void warp_rows_each_logit(const float *__restrict__ logits, int row0, int T, int Nr,
+                                                     float (*blk)[33], int lane, F &&f) {
+    for (int c0 = 0; c0 < Nr; c0 += 32) {
+        const int c = c0 + lane;
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+            const int row = row0 + r;
+            blk[r][lane] = (row < T && c < Nr) ? __ldg(logits + (size_t)row * Nr + c) : 0.0f;
+        }
+        __syncwarp();
+        const int cn = min(32, Nr - c0);
+        for (int j = 0; j < cn; ++j) f(c0 + j, blk[lane][j]);
+        __syncwarp();
     }
 }
 
@@ -75,6 +99,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
     __shared__ float bias_s[kMaxExperts];
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
+    __shared__ float blocks[kWarpsPerCta][32][33];  // per-warp transpose buffer (padded: no bank conflicts)
 
     for (int i = threadIdx.x; i < Nr; i += kThreads) {
         bias_s[i] = bias[i];
@@ -84,42 +109,46 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
     __syncthreads();
 
     const bool want_tiles = tile_counts != nullptr;
-    const bool vec4 = (Nr & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
     int *hist = want_tiles ? hist_tile : hist_total;
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    float(*blk)[33] = blocks[warp];
 
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int row = tile * kTileTokens + threadIdx.x;
-        if (row < T) {
-            const float *x = logits + (size_t)row * Nr;
+        const int row0 = tile * kTileTokens + warp * 32;
+        const int row = row0 + lane;
+        if (row0 < T) {  // warp-uniform: the whole warp joins the block loads
             // pass 1: approximate keys, their K-th largest
-            RowTopK<K> approx;
+            TopValues<K> approx;
             approx.init();
-            for_each_logit(x, Nr, vec4, [&](int c, float xv) {
-                approx.push(__fadd_rn(sigmoid_fast(xv), bias_s[c]), 0.0f, c);
+            warp_rows_each_logit(logits, row0, T, Nr, blk, lane, [&](int c, float xv) {
+                approx.push(__fadd_rn(sigmoid_fast(xv), bias_s[c]));
             });
-            const float tau = approx.key[K - 1];
+            const float tau = approx.v[K - 1];
             // |approximate key - exact key| <= kSigmaErr + one rounding of each add
             const float lim = tau - 2.0f * (kSigmaErr + 2.384185791015625e-7f * fabsf(tau));
             // pass 2: exact keys of the candidates only
             RowTopK<K> tk;
             tk.init();
-            for_each_logit(x, Nr, vec4, [&](int c, float xv) {
+            warp_rows_each_logit(logits, row0, T, Nr, blk, lane, [&](int c, float xv) {
                 if (__fadd_rn(sigmoid_fast(xv), bias_s[c]) >= lim) {
                     const float s = sigmoid_rounded_once(xv);
                     tk.push(__fadd_rn(s, bias_s[c]), s, c);
                 }
             });
-            double sum = 0.0;
+            if (row < T) {
+                double sum = 0.0;
 #pragma unroll
-            for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)tk.score[k]);
-            int32_t *oi = topk_idx + (size_t)row * K;
-            float *og = gates + (size_t)row * K;
+                for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)tk.score[k]);
+                int32_t *oi = topk_idx + (size_t)row * K;
+                float *og = gates + (size_t)row * K;
 #pragma unroll
-            for (int k = 0; k < K; ++k) {
-                oi[k] = tk.idx[k];
-                og[k] = __double2float_rn(__ddiv_rn((double)tk.score[k], sum));
-                if ((unsigned)tk.idx[k] < (unsigned)Nr) atomicAdd(&hist[tk.idx[k]], 1);
+                for (int k = 0; k < K; ++k) {
+                    oi[k] = tk.idx[k];
+                    og[k] = __double2float_rn(__ddiv_rn((double)tk.score[k], sum));
+                    if ((unsigned)tk.idx[k] < (unsigned)Nr) atomicAdd(&hist[tk.idx[k]], 1);
+                }
             }
         }
         if (want_tiles) {
