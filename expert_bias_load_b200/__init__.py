@@ -45,6 +45,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "ebl_strerror": (ctypes.c_char_p, [_I]),
     "ebl_version": (_I, []),
+    "ebl_last_cuda_error": (ctypes.c_char_p, []),
     "ebl_tile_tokens": (_I, []),
     "router_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "router_forward_zloss": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
@@ -65,6 +66,8 @@ class EblError(RuntimeError):
     def __init__(self, fn, code):
         self.code = code
         text = lib().ebl_strerror(code).decode() if _lib is not None else str(code)
+        if code == EBL_ECUDA and _lib is not None:
+            text += "; " + lib().ebl_last_cuda_error().decode()
         super().__init__("%s failed: %d (%s)" % (fn, code, text))
 
 

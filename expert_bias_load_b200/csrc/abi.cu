@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -26,7 +27,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-int cuda_fail() {
+// The last CUDA failure this thread saw inside the library (for ebl_last_cuda_error).
+thread_local char g_last_error[160] = "none";
+
+void record_error(const char *where, const char *what) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s", where, what);
+}
+
+int cuda_fail(const char *where, cudaError_t e) {
+    record_error(where, cudaGetErrorString(e));
     (void)cudaGetLastError();  // clear a sticky launch error so the caller's context stays usable
     return EBL_ECUDA;
 }
@@ -39,14 +48,17 @@ struct DeviceInfo {
 // SM count and the internal status address of the current device (cached).
 int device_info(DeviceInfo *out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail();
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     if (dev < 0 || dev >= kMaxDevices) return EBL_EUNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mu);
     if (g_num_sms[dev] == 0) {
         int sms = 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return cuda_fail();
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_internal_status) != cudaSuccess) return cuda_fail();
+        e = cudaGetSymbolAddress(&p, g_internal_status);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress", e);
         g_status_ptr[dev] = static_cast<int32_t *>(p);
         g_num_sms[dev] = sms;
     }
@@ -60,9 +72,12 @@ int get_encoder() {
     if (g_encode) return EBL_OK;
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || fn == nullptr)
-        return cuda_fail();
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDriverEntryPoint", e);
+    if (q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        record_error("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled not found");
+        return EBL_ECUDA;
+    }
     g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     return EBL_OK;
 }
@@ -76,7 +91,13 @@ int encode_bf16_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t c
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? EBL_OK : EBL_ECUDA;
+    if (r != CUDA_SUCCESS) {
+        char msg[64];
+        snprintf(msg, sizeof msg, "CUresult %d", (int)r);
+        record_error("cuTensorMapEncodeTiled", msg);
+        return EBL_ECUDA;
+    }
+    return EBL_OK;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -117,7 +138,7 @@ int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const flo
     cudaError_t e = ebl::launch_router_gemm(th, tw, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts,
                                             zloss_sum, status ? status : di.internal_status, di.num_sms,
                                             reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 }  // namespace
@@ -142,6 +163,8 @@ const char *ebl_strerror(int code) {
 }
 
 int ebl_version(void) { return 10000; }
+
+const char *ebl_last_cuda_error(void) { return g_last_error; }
 
 int ebl_tile_tokens(void) { return ebl::kTileTokens; }
 
@@ -175,7 +198,7 @@ int router_forward_logits(const float *logits, const float *bias, int T, int N_r
     if (rc) return rc;
     cudaError_t e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts,
                                               di.num_sms, reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 int smebu_step_layers(int32_t *counts, float *bias, float *momentum, int L, int N_r, float lambda, float beta,
@@ -191,7 +214,7 @@ int smebu_step_layers(int32_t *counts, float *bias, float *momentum, int L, int 
     cudaError_t e = ebl::launch_smebu(counts, bias, momentum, L, N_r, lambda, beta, kappa, linear, reset_counts,
                                       maxvio_out, status ? status : di.internal_status,
                                       reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 int smebu_step(int32_t *counts, float *bias, float *momentum, int N_r, float lambda, float beta, float kappa,
@@ -211,7 +234,7 @@ int sign_update_step(int32_t *counts, float *bias, int N_r, float gamma, int res
     cudaError_t e = ebl::launch_sign_update(counts, bias, N_r, gamma, reset_counts, maxvio_out,
                                             status ? status : di.internal_status,
                                             reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 size_t ebl_dispatch_workspace_bytes(int T, int N_r) {
@@ -236,12 +259,12 @@ int moe_dispatch(const uint16_t *hidden, const int32_t *topk_idx, const int32_t 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (T == 0) {  // offsets of an empty batch are all zero
         cudaError_t e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (size_t)(N_r + 1), st);
-        return e == cudaSuccess ? EBL_OK : cuda_fail();
+        return e == cudaSuccess ? EBL_OK : cuda_fail("cudaMemsetAsync", e);
     }
     cudaError_t e = ebl::launch_dispatch(hidden, topk_idx, tile_counts, T, d, N_r, K, offsets, perm, dest,
                                          dispatched, workspace, status ? status : di.internal_status, di.num_sms,
                                          st);
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *dest, int T, int d, int K,
@@ -258,7 +281,7 @@ int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *d
     cudaError_t e = ebl::launch_combine(expert_out, gates, dest, T, d, K, out,
                                         status ? status : di.internal_status, di.num_sms,
                                         reinterpret_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? EBL_OK : cuda_fail();
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 int ebl_read_internal_status(int32_t *out, int clear) {
@@ -266,9 +289,9 @@ int ebl_read_internal_status(int32_t *out, int clear) {
     DeviceInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
-    if (cudaMemcpy(out, di.internal_status, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
-        return cuda_fail();
-    if (clear && cudaMemset(di.internal_status, 0, sizeof(int32_t)) != cudaSuccess) return cuda_fail();
+    cudaError_t e = cudaMemcpy(out, di.internal_status, sizeof(int32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpy", e);
+    if (clear && (e = cudaMemset(di.internal_status, 0, sizeof(int32_t))) != cudaSuccess) return cuda_fail("cudaMemset", e);
     return EBL_OK;
 }
 

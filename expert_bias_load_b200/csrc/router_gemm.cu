@@ -33,6 +33,8 @@
 // expert per CTA; tile_counts with one store per expert per tile.  Every
 // pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
 
+#include <mutex>
+
 #include "launch.h"
 #include "ptx.cuh"
 #include "topk.cuh"
@@ -486,6 +488,57 @@ int stages_for(int Nr, int K, int G) {  // the layout is the same with and witho
     return s;
 }
 
+// Per device and kernel instantiation: the largest dynamic shared-memory size
+// granted so far (the attribute is a limit, so it only ever grows), and per
+// shared-memory size the number of co-resident clusters.  Set up on first use
+// only, so that later launches (for instance inside a CUDA graph capture)
+// issue nothing but the launch itself.
+struct SmemGrant {
+    const void *kern;
+    int device;
+    size_t smem;
+};
+struct ClusterFit {
+    const void *kern;
+    int device;
+    size_t smem;
+    int clusters;
+};
+std::mutex g_setup_mu;
+SmemGrant g_grant[128];
+int g_num_grant = 0;
+ClusterFit g_fit[256];
+int g_num_fit = 0;
+
+cudaError_t launch_setup(const void *kern, size_t smem, cudaLaunchConfig_t *cfg, int *clusters) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(g_setup_mu);
+    int gi = -1;
+    for (int i = 0; i < g_num_grant; ++i)
+        if (g_grant[i].kern == kern && g_grant[i].device == dev) gi = i;
+    if (gi < 0 || g_grant[gi].smem < smem) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        if (gi >= 0)
+            g_grant[gi].smem = smem;
+        else if (g_num_grant < 128)
+            g_grant[g_num_grant++] = {kern, dev, smem};
+    }
+    for (int i = 0; i < g_num_fit; ++i)
+        if (g_fit[i].kern == kern && g_fit[i].device == dev && g_fit[i].smem == smem) {
+            *clusters = g_fit[i].clusters;
+            return cudaSuccess;
+        }
+    int active = 0;  // clusters that fit on the device at once
+    if (cudaOccupancyMaxActiveClusters(&active, kern, cfg) != cudaSuccess) active = 0;
+    (void)cudaGetLastError();
+    if (g_num_fit < 256) g_fit[g_num_fit++] = {kern, dev, smem, active};
+    *clusters = active;
+    return cudaSuccess;
+}
+
 template <int K, int G>
 cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
                       int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zloss_sum,
@@ -493,8 +546,6 @@ cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float 
     auto kern = zloss_sum ? router_gemm_kernel<K, G, true> : router_gemm_kernel<K, G, false>;
     const int stages = stages_for(Nr, K, G);
     const size_t smem = 1024 + misc_layout(Nr, K, G, stages).total;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     const int num_work = (num_tiles + kPair - 1) / kPair;
     int units = num_sms / kPair;
@@ -510,10 +561,10 @@ cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float 
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.gridDim = dim3(kPair * units, 1, 1);
-    int active = 0;  // clusters that fit on the device at once
-    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0 && active < units)
-        units = active;
-    (void)cudaGetLastError();
+    int active = 0;
+    cudaError_t err = launch_setup(reinterpret_cast<const void *>(kern), smem, &cfg, &active);
+    if (err != cudaSuccess) return err;
+    if (active > 0 && active < units) units = active;
     if (units > num_work) units = num_work;
     cfg.gridDim = dim3(kPair * units, 1, 1);
     err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, zloss_sum,

@@ -69,6 +69,11 @@ const char *ebl_strerror(int code);
 /* Library version, major*10000 + minor*100 + patch. */
 int ebl_version(void);
 
+/* The last CUDA failure behind an EBL_ECUDA return on the calling thread, as
+ * "call: reason" text ("none" if there was none).  Never NULL; valid until the
+ * next library call on this thread. */
+const char *ebl_last_cuda_error(void);
+
 /* Tokens per router tile: the row count of one tile_counts row (128). */
 int ebl_tile_tokens(void);
 

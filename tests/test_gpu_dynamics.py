@@ -1,0 +1,130 @@
+"""Multi-step balancing runs on the mid and drift workloads (GEMM mode, full
+size) and a CUDA-graph capture of the router step.
+
+The pages give no numbers for the dynamics (SMEBU settles, the sign update
+keeps oscillating at +-gamma, a linear update goes unstable), so these tests
+assert only what the equations fix -- sum of b stays at its start value under
+SMEBU (the step is re-centred) and at 0 under the sign update (b is
+re-centred), |m| <= 2 lambda, the loads add up to K*T -- and print the MaxVio
+trajectories (pytest -s) as the workloads ask.
+"""
+import json
+import math
+
+import pytest
+import torch
+
+import expert_bias_load_b200 as ebl
+import synth
+from expert_bias_load_b200.telemetry import maxvio_level, step_stats
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(h_of_step, W, K, steps, update, gamma=1e-3):
+    dev = W.device
+    Nr = W.shape[0]
+    b = torch.zeros(Nr, device=dev)
+    m = torch.zeros(Nr, device=dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    mv = torch.zeros(1, device=dev)
+    traj = []
+    for s in range(steps):
+        h = h_of_step(s)
+        ebl.router_forward(h, W, b, K, counts)
+        prev = b.clone()
+        c = counts.clone()
+        if update == "smebu":
+            ebl.smebu_step(counts, b, m, reset_counts=True, maxvio=mv)
+        else:
+            ebl.sign_update_step(counts, b, gamma, reset_counts=True, maxvio=mv)
+        st = step_stats(c, b, m if update == "smebu" else None, mv, prev)
+        assert st["total_load"] == K * h.shape[0]
+        traj.append(st)
+    return traj, b, m
+
+
+def test_mid_workload_sign_vs_smebu(cuda_device):
+    cfg = synth.WORKLOADS["mid"]
+    T, d, Nr, K, steps = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"], cfg["steps"]
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(cuda_device)
+    hs = lambda s: synth.hidden_normal(T, d, seed=synth.step_seed("mid", s), device=cuda_device)
+    tr_smebu, b1, m1 = _run(hs, W, K, steps, "smebu")
+    tr_sign, b2, _ = _run(hs, W, K, steps, "sign")
+    for st in tr_smebu:
+        assert abs(st["bias_sum"]) <= 1e-4                   # b0 = 0 and every step sums to 0
+        assert st["momentum_absmax"] <= 2 * 5e-4 * (1 + 1e-6)
+    for st in tr_sign:
+        assert abs(st["bias_sum"]) <= 1e-4                   # b is re-centred every step
+        assert st["bias_step_absmax"] <= 2 * 1e-3 * (1 + 1e-6)
+    print("\nmid workload MaxVio per step")
+    print(json.dumps({"smebu": [round(s["maxvio"], 3) for s in tr_smebu],
+                      "sign": [round(s["maxvio"], 3) for s in tr_sign]}))
+
+
+def test_drift_workload_smebu_200_steps(cuda_device):
+    cfg = synth.WORKLOADS["drift"]
+    T, d, Nr, K, steps = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"], cfg["steps"]
+    dev = cuda_device
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    # the smallest drift strength on the scan that starts with MaxVio > 6
+    mu = None
+    for cand in (0.5, 1.0, 2.0, 4.0, 8.0):
+        h = synth.hidden_drift(T, d, W, seed=synth.step_seed("drift", 0), mu=cand, device=dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        ebl.router_forward(h, W, torch.zeros(Nr, device=dev), K, counts)
+        c = counts.double()
+        mv0 = math.inf if float(c.min()) == 0 else float(c.max() / c.min())
+        if mv0 > 6:
+            mu = cand
+            break
+    assert mu is not None, "no drift strength on the scan gives MaxVio > 6"
+    hs = lambda s: synth.hidden_drift(T, d, W, seed=synth.step_seed("drift", s), mu=mu, device=dev)
+    tr, b, m = _run(hs, W, K, steps, "smebu")
+    assert maxvio_level(tr[0]["maxvio"]) == "alarm"
+    for st in tr:
+        assert abs(st["bias_sum"]) <= 1e-4
+        assert st["momentum_absmax"] <= 2 * 5e-4 * (1 + 1e-6)
+    print("\ndrift workload mu=%g MaxVio every 10 steps" % mu)
+    print(json.dumps([round(tr[i]["maxvio"], 3) for i in range(0, steps, 10)] + [round(tr[-1]["maxvio"], 3)]))
+
+
+def test_router_step_in_cuda_graph(cuda_device):
+    """The router step (GEMM-mode router, SMEBU with reset) captured once in a
+    CUDA graph and replayed gives the same state as eager launches."""
+    dev = cuda_device
+    T, d, Nr, K = 4096, 512, 256, 4
+    W = synth.router_weight(Nr, d, seed=9).to(dev)
+    h = synth.hidden_normal(T, d, seed=10, device=dev)
+    state = {}
+    for mode in ("eager", "graph"):
+        b = synth.dead_start_bias(Nr, device=dev)
+        m = torch.zeros(Nr, device=dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        g = torch.empty(T, K, device=dev)
+        mv = torch.zeros(1, device=dev)
+
+        def step(stream=None):
+            ebl.router_forward(h, W, b, K, counts, topk_idx=idx, gates=g, stream=stream)
+            ebl.smebu_step(counts, b, m, reset_counts=True, maxvio=mv, stream=stream)
+
+        if mode == "eager":
+            for _ in range(5):
+                step()
+        else:
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                step(s)                               # warm-up launch outside the graph
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(torch.cuda.current_stream())
+            for _ in range(4):
+                graph.replay()
+        torch.cuda.synchronize()
+        state[mode] = (b.clone(), m.clone(), idx.clone(), g.clone())
+    for a, c in zip(state["eager"], state["graph"]):
+        assert torch.equal(a, c)

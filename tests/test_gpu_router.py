@@ -168,3 +168,18 @@ def test_router_zloss_vs_oracle(cuda_device, T, d, Nr, K):
     ebl.router_forward_zloss(h, W, bias, K, c2, z)
     torch.cuda.synchronize()
     assert abs(float(z.item()) - 2 * ref) <= 2e-4 * ref
+
+
+def test_alternating_shapes_share_one_kernel(cuda_device):
+    """Shapes that need different shared-memory sizes on the same kernel
+    instantiation, in both orders (the larger one first, then a smaller one,
+    then the larger one again), all launch."""
+    dev = cuda_device
+    for Nr in (64, 256, 64, 128, 256, 64):
+        T, d, K = 300, 256, 4
+        h = synth.hidden_normal(T, d, seed=Nr, device=dev)
+        W = synth.router_weight(Nr, d, seed=Nr + 1).to(dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        idx, g = ebl.router_forward(h, W, torch.zeros(Nr, device=dev), K, counts)
+        torch.cuda.synchronize()
+        assert int(counts.sum().item()) == T * K
