@@ -49,6 +49,7 @@ __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f,
 constexpr float kSigmaErr = 4.0e-6f;
 
 constexpr int kWarpsPerCta = kThreads / 32;
+constexpr int kMaxCand = 8;  // candidates a lane buffers before scoring them exactly
 
 // The K largest values seen so far (with repeats), sorted descending; one
 // fmax/fmin pair per slot and value, no branches.  NaN values are dropped.
@@ -100,6 +101,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
     __shared__ float blocks[kWarpsPerCta][32][33];  // per-warp transpose buffer (padded: no bank conflicts)
+    __shared__ float cand_x[kWarpsPerCta][kMaxCand][32];  // per-lane candidates of pass 2: logit, expert
+    __shared__ int cand_c[kWarpsPerCta][kMaxCand][32];
 
     for (int i = threadIdx.x; i < Nr; i += kThreads) {
         bias_s[i] = bias[i];
@@ -128,15 +131,30 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
             const float tau = approx.v[K - 1];
             // |approximate key - exact key| <= kSigmaErr + one rounding of each add
             const float lim = tau - 2.0f * (kSigmaErr + 2.384185791015625e-7f * fabsf(tau));
-            // pass 2: exact keys of the candidates only
+            // pass 2: exact keys of the candidates only.  Candidates are buffered
+            // per lane (in increasing expert index) and scored after the scan,
+            // so the fp64 work runs in a short loop instead of under a branch
+            // that some lane of the warp takes at most experts.
             RowTopK<K> tk;
             tk.init();
-            warp_rows_each_logit(logits, row0, T, Nr, blk, lane, [&](int c, float xv) {
-                if (__fadd_rn(sigmoid_fast(xv), bias_s[c]) >= lim) {
-                    const float s = sigmoid_rounded_once(xv);
+            int nc = 0;
+            auto flush = [&]() {
+                for (int q = 0; q < nc; ++q) {
+                    const int c = cand_c[warp][q][lane];
+                    const float s = sigmoid_rounded_once(cand_x[warp][q][lane]);
                     tk.push(__fadd_rn(s, bias_s[c]), s, c);
                 }
+                nc = 0;
+            };
+            warp_rows_each_logit(logits, row0, T, Nr, blk, lane, [&](int c, float xv) {
+                if (__fadd_rn(sigmoid_fast(xv), bias_s[c]) >= lim) {
+                    if (nc == kMaxCand) flush();  // many near-equal keys: score what we have first
+                    cand_x[warp][nc][lane] = xv;
+                    cand_c[warp][nc][lane] = c;
+                    ++nc;
+                }
             });
+            flush();
             if (row < T) {
                 double sum = 0.0;
 #pragma unroll

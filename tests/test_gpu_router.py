@@ -183,3 +183,19 @@ def test_alternating_shapes_share_one_kernel(cuda_device):
         idx, g = ebl.router_forward(h, W, torch.zeros(Nr, device=dev), K, counts)
         torch.cuda.synchronize()
         assert int(counts.sum().item()) == T * K
+
+
+def test_logits_mode_all_equal_keys(cuda_device):
+    """Every expert has the same key (logits 0, bias 0), and rows where 40
+    experts share the top key: the candidate buffer overflows and is scored in
+    several rounds, and the lowest indices still win."""
+    T, Nr, K = 200, 256, 4
+    x = torch.zeros(T, Nr)
+    bias = torch.zeros(Nr)
+    x[100:, 60:100] = 1.0                          # rows 100.. : experts 60..99 tie at the top
+    idx, gates, counts, tiles = _run_logits(x, bias, K)
+    assert np.array_equal(idx[:100], np.tile(np.arange(K, dtype=np.int32), (100, 1)))
+    assert np.array_equal(idx[100:], np.tile(np.arange(60, 60 + K, dtype=np.int32), (100, 1)))
+    assert np.all(gates == np.float32(0.25))
+    ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx) and np.array_equal(counts, ref.counts)
