@@ -21,14 +21,15 @@
 //               K=16, 8 per stage) for the pair into a double-buffered
 //               fp32 accumulator (2 x N_r columns per CTA), so the epilogue of
 //               tile i overlaps the MMAs of tile i+1.
-//   epilogue    G = 2 (or 1) groups of 4 warps.  Warp w reads TMEM lane quadrant w%4 (one
-//               token row per thread); group g = w/4 owns the experts
-//               [g*N_r/G, (g+1)*N_r/G).  Each thread runs sigmoid, +bias and a
-//               running Top-K over its experts; groups 1..G-1 hand their
-//               sorted partial lists to group 0 through shared memory, and
-//               group 0 merges them, writes indices and gates, and keeps the
-//               load histogram.  Splitting the experts puts G epilogue warps on
-//               every SM sub-partition, which hides the epilogue's latencies.
+//   epilogue    G groups of 4 warps (G = 2 when N_r % 64 == 0, else 1).  Warp
+//               w reads TMEM lane quadrant w%4 (one token row per thread);
+//               group g = w/4 owns the experts [g*N_r/G, (g+1)*N_r/G).  Each
+//               thread runs sigmoid, +bias and a running Top-K over its
+//               experts; group 1 hands its sorted partial list to group 0
+//               through shared memory, and group 0 merges, writes indices and
+//               gates, and keeps the load histogram (and, for the z-loss, a
+//               running log-sum-exp per row).  Two epilogue warps per SM
+//               sub-partition keep up with the MMAs.
 // The logits never leave TMEM.  Counts reach global memory with one atomic per
 // expert per CTA; tile_counts with one store per expert per tile.  Every
 // pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
@@ -42,12 +43,12 @@
 namespace ebl {
 namespace {
 
-constexpr int kSubK = 64;                // hidden elements per TMA box: one 128-byte swizzle row
-constexpr int kNSub = 2;                 // boxes per pipeline stage
-constexpr int kBlockK = kSubK * kNSub;   // hidden elements per stage (8 MMAs between barriers)
-constexpr int kUmmaK = 16;   // K of one kind::f16 MMA
-constexpr int kChunk = 16;   // TMEM columns per epilogue load
-constexpr int kMaxStages = 8;
+constexpr int kSubK = 64;               // hidden elements per TMA box: one 128-byte swizzle row
+constexpr int kNSub = 2;                // boxes per pipeline stage
+constexpr int kBlockK = kSubK * kNSub;  // hidden elements per stage (8 MMAs between barriers)
+constexpr int kUmmaK = 16;              // K of one kind::f16 MMA
+constexpr int kChunk = 16;              // TMEM columns per epilogue load
+constexpr int kMaxStages = 8;           // ring depth cap (shared memory decides: 3 at N_r = 256)
 constexpr uint32_t kASubBytes = kTileTokens * kSubK * 2;
 constexpr uint32_t kATileBytes = kASubBytes * kNSub;
 
