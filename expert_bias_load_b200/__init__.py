@@ -59,6 +59,7 @@ SIGNATURES = {
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "ebl_read_internal_status": (_I, [_P, _I]),
     "ebl_selftest_wait_timeout": (_I, [_P, ctypes.c_uint, _P]),
+    "ebl_selftest_score_error": (_I, [_P, ctypes.c_int64, _P, _P, _P]),
 }
 
 
@@ -279,3 +280,16 @@ def selftest_wait_timeout(status, limit_us=20000, stream=None):
     """Run the bounded-wait self-test; EBL_ST_TIMEOUT lands in status (int32 [1])."""
     _check(status, "status", torch.int32, (1,))
     _call("ebl_selftest_wait_timeout", _ptr(status), int(limit_us), _stream(stream))
+
+
+def selftest_score_error(x, max_err=None, stream=None):
+    """Largest distance between the approximate score logits mode ranks with
+    and the exact one over the fp32 values in x (device), and the error bound
+    that ranking assumes.  Returns (max_err as a float, bound)."""
+    _check(x, "x", torch.float32)
+    if max_err is None:
+        max_err = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(max_err, "max_err", torch.float32, (1,))
+    bound = ctypes.c_float(0.0)
+    _call("ebl_selftest_score_error", _ptr(x), int(x.numel()), _ptr(max_err), ctypes.c_void_p(ctypes.addressof(bound)), _stream(stream))
+    return float(max_err.item()), float(bound.value)

@@ -8,23 +8,26 @@
 // Sources: "Arcee Trinity Large Technical Report" section 2.3; "SMEBU Load
 // Balancing" eq. (17).
 //
-// Layout: one thread per token row (a CTA of 128 threads takes a 128-token
-// tile; persistent grid).  A warp's 32 rows are read together, 32 experts at a
-// time: each load instruction fetches 128 contiguous bytes of one row, and the
-// 32 x 32 block is transposed through padded shared memory so that every thread
-// then walks its own row in increasing expert index.  Each thread keeps a
-// running Top-K in registers; visiting experts in increasing index lets a
-// strict comparison keep the lower index first on equal keys.  A shared-memory
-// histogram is flushed per tile (tile_counts) and per CTA (counts).
+// The fp64 sigmoid is only evaluated where it can matter.  An approximate key
+// with a bounded distance to the exact one ranks all experts; the K-th largest
+// approximate key tau bounds the exact K-th key, and only experts whose
+// approximate key is within twice that distance of tau can be in the exact
+// Top-K.  Those candidates (usually K or K+1 per token) are scored exactly and
+// the exact Top-K is taken among them: the same result as scoring every expert
+// in fp64.
 //
-// The fp64 sigmoid is only evaluated where it can matter.  A first pass ranks
-// the experts with an fp32 sigmoid whose distance to the fp64-rounded value
-// is bounded (kSigmaErr); its K-th key tau bounds the exact K-th key within
-// kSigmaErr plus the rounding of the key add.  Only experts whose approximate
-// key is within twice that margin of tau can be in the exact Top-K, so the
-// second pass computes the exact score of those candidates alone (usually K or
-// K+1 of them) and selects among them: the same result as evaluating every
-// expert in fp64.
+// Two kernels.  The vector kernel (N_r % 4 == 0, 16-byte aligned logits, the
+// usual case) gives each token row to 8 lanes: every load instruction fetches
+// 128 contiguous bytes of each of 4 rows, a lane's 4*NV logits and their keys
+// stay in registers, tau comes from a butterfly over the 8 lanes, and the
+// candidates are compacted per row in shared memory, scored by the row's 8
+// lanes and ranked in parallel.  The logits are read from HBM exactly once.
+// The row kernel (any N_r, 4-byte alignment) gives each row to one thread and
+// reads the logits twice.
+
+#include <cfloat>
+#include <cstdint>
+#include <mutex>
 
 #include "launch.h"
 #include "ptx.cuh"
@@ -38,7 +41,7 @@ constexpr int kThreads = kTileTokens;  // one thread per row of a tile
 __device__ __forceinline__ float sigmoid_rounded_once(float x) {
     // fp64 evaluation, one rounding to fp32 at the end
     const double e = exp(-(double)x);
-    return __double2float_rn(__ddiv_rn(1.0, __dadd_rn(1.0, e)));
+    return __double2float_rn(__drcp_rn(__dadd_rn(1.0, e)));  // correctly rounded 1/y, the same as 1.0/y
 }
 
 // fp32 sigmoid from the fast intrinsics: __expf (at most 2 + 1.173|x| ulp off)
@@ -66,6 +69,29 @@ struct TopValues {
             const float hi = fmaxf(v[k], x);
             x = fminf(v[k], x);
             v[k] = hi;
+        }
+    }
+    // Keep the K largest of this lane's list and lane (lane ^ m)'s (K a power
+    // of two): the elementwise max of one list and the other reversed is a
+    // bitonic sequence holding the K largest of both, which a half-cleaner
+    // cascade sorts.
+    __device__ __forceinline__ void merge_xor(int m) {
+        static_assert((K & (K - 1)) == 0, "bitonic merge needs a power-of-two list");
+        float o[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) o[k] = __shfl_xor_sync(0xffffffffu, v[k], m);
+#pragma unroll
+        for (int k = 0; k < K; ++k) v[k] = fmaxf(v[k], o[K - 1 - k]);
+#pragma unroll
+        for (int h = K / 2; h > 0; h >>= 1) {
+#pragma unroll
+            for (int i = 0; i < K; ++i) {
+                if ((i & h) == 0) {
+                    const float a = v[i], b = v[i + h];
+                    v[i] = fmaxf(a, b);
+                    v[i + h] = fminf(a, b);
+                }
+            }
         }
     }
 };
@@ -185,12 +211,451 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
         if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
 }
 
+
+// ---------------------------------------------------------------------------
+// Vector kernel: 8 lanes per token row, one HBM read of the logits.
+// ---------------------------------------------------------------------------
+
+constexpr int kLanesPerRow = 8;
+constexpr int kRowsPerGroup = 32 / kLanesPerRow;         // rows a warp takes at once
+constexpr int kGroupsPerWarp = 32 / kRowsPerGroup;       // row groups of a warp per tile
+constexpr int kWin = 32;                                 // candidates of a row scored per round
+constexpr int kWinPad = kWin + 1;                        // odd stride: rows of a group hit different banks
+
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Approximate key from hb = fl(0.5 + b): 0.5 tanh(x/2) + 0.5 + b is
+// sigmoid(x) + b.  Distance to the exact key fl(fl(sigmoid(x)) + b):
+//   0.5 |tanh.approx(x/2) - tanh(x/2)|   about 2^-12 (tanh.approx.f32's relative
+//                                        error is about 2^-11; measured by
+//                                        ebl_selftest_score_error)
+//   fl(sigmoid(x)) - sigmoid(x)          <= 2^-25
+//   roundings of hb, the fma, the add    <= 2^-24 (|hb| + |key_a| + |key_e|)
+//                                        <= 2^-24 (3 |key_e| + 1.5) + O(2^-36)
+// (|b| <= |key_e| + 1), so |key_a - key_e| <= kKeyErr + 2^-22 |key_e| with the
+// constant part given an 8x margin.
+constexpr float kKeyErr = 0x1p-9f;
+__device__ __forceinline__ float key_approx(float x, float hb) { return fmaf(0.5f, tanh_approx(0.5f * x), hb); }
+
+// Lower limit on the approximate key of every member of the exact Top-K, from
+// tau' <= the K-th largest approximate key.  With E(y) = kKeyErr + 2^-22 |y|:
+// the K-th exact key tau_e satisfies tau' <= tau_e + E(tau_e), so
+// tau_e >= tau' - kKeyErr - 2^-21 |tau' - kKeyErr|; a member i has
+// key_a >= key_e - E(key_e) >= tau_e - E(tau_e).  Together (and with the
+// rounding of this fp32 expression) key_a >= tau' - 2 kKeyErr - 2^-19 |tau'|.
+// An empty list (tau' = -inf) admits every finite key; padding keys (-inf)
+// never pass.
+__device__ __forceinline__ float candidate_limit(float tau) {
+    return fmaxf(tau - (2.0f * kKeyErr + 0x1p-19f * fabsf(tau)), -FLT_MAX);
+}
+
+constexpr int kStages = 2;  // row groups of a warp in the shared-memory ring: one loads while one is ranked
+
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src, bool pred) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    const int n = pred ? 16 : 0;  // 0: the 16 bytes are zero-filled and nothing is read
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// dynamic shared memory of the vector kernel: the logits ring
+template <int NV>
+constexpr size_t vec_ring_bytes() {
+    return sizeof(float) * kWarpsPerCta * kStages * kRowsPerGroup * 32 * NV;
+}
+
+template <int K, int NV>
+__global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float *__restrict__ logits,
+                                                                     const float *__restrict__ bias, int T, int Nr,
+                                                                     int32_t *__restrict__ topk_idx,
+                                                                     float *__restrict__ gates,
+                                                                     int32_t *__restrict__ counts,
+                                                                     int32_t *__restrict__ tile_counts) {
+    // lane-local lists of the approximate pass hold P >= K values (P a power of two)
+    constexpr int P = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
+    constexpr int kRow = 32 * NV;  // floats per row in the ring (N_r rounded up, zero-filled)
+    static_assert(NV % 2 == 0 && kRow <= kMaxExperts, "a lane holds NV float4 of a row, in pairs");
+    extern __shared__ __align__(16) float ring_s[];  // [warp][stage][row of group][kRow]
+    __shared__ __align__(16) float hb_s[kMaxExperts];  // fl(0.5 + b); -inf past N_r
+    __shared__ float bias_s[kMaxExperts];
+    __shared__ int hist_total[kMaxExperts];
+    __shared__ int hist_tile[kMaxExperts];
+    __shared__ int cand_c[kWarpsPerCta][kRowsPerGroup][kWinPad];  // a round's candidates of each row
+    __shared__ float cand_key[kWarpsPerCta][kRowsPerGroup][kWinPad];
+    __shared__ float cand_s[kWarpsPerCta][kRowsPerGroup][kWinPad];
+    __shared__ float sel_key[kWarpsPerCta][kRowsPerGroup][2 * K];  // [0,K): the Top-K so far; [K,2K): a later round's
+    __shared__ float sel_s[kWarpsPerCta][kRowsPerGroup][2 * K];
+    __shared__ int sel_c[kWarpsPerCta][kRowsPerGroup][2 * K];
+
+    for (int i = threadIdx.x; i < kMaxExperts; i += kThreads) {
+        const bool in = i < Nr;
+        const float b = in ? bias[i] : 0.0f;
+        bias_s[i] = b;
+        hb_s[i] = in ? __fadd_rn(0.5f, b) : -INFINITY;
+        hist_total[i] = 0;
+        hist_tile[i] = 0;
+    }
+    for (int i = threadIdx.x; i < kWarpsPerCta * kRowsPerGroup * 2 * K; i += kThreads) {
+        (&sel_key[0][0][0])[i] = -INFINITY;
+        (&sel_s[0][0][0])[i] = 0.0f;
+        (&sel_c[0][0][0])[i] = 0;
+    }
+    __syncthreads();
+
+    const bool want_tiles = tile_counts != nullptr;
+    int *hist = want_tiles ? hist_tile : hist_total;
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int r = lane >> 3;  // row of the group this lane works on
+    const int j = lane & 7;   // lane within the row: float4 columns j, j + 8, j + 16, ...
+    float *ring = ring_s + (size_t)warp * kStages * kRowsPerGroup * kRow;
+    int *cc = cand_c[warp][r];
+    float *ck = cand_key[warp][r];
+    float *cs = cand_s[warp][r];
+    float *sk = sel_key[warp][r];
+    float *ss = sel_s[warp][r];
+    int *sc = sel_c[warp][r];
+
+    // Work item i of this warp: row group i % 8 of tile blockIdx.x + (i / 8) * gridDim.x.
+    // Its 4 rows go to ring stage i % kStages; lane j of a row copies float4
+    // columns 8m + j, so each copy instruction covers 128 contiguous bytes of
+    // each of the 4 rows.  Rows past T are zero-filled without a read.
+    auto item_row = [&](int item) -> int64_t {
+        const int64_t tile = (int64_t)blockIdx.x + (int64_t)(item >> 3) * gridDim.x;
+        return tile * kTileTokens + warp * 32 + (item & 7) * kRowsPerGroup + r;
+    };
+    auto issue = [&](int item) {
+        const int64_t row = item_row(item);
+        const bool rin = row < T;
+        const float *src = logits + (rin ? row : 0) * (int64_t)Nr;
+        float *dst = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+            const int c = 4 * (8 * m + j);
+            const bool ok = rin && c < Nr;
+            cp_async_16(dst + c, src + (ok ? c : 0), ok);
+        }
+        cp_async_commit();
+    };
+
+    const int items = num_tiles > (int)blockIdx.x
+                          ? ((num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * kGroupsPerWarp
+                          : 0;
+#pragma unroll
+    for (int q = 0; q < kStages - 1; ++q) issue(q);
+    for (int item = 0; item < items; ++item) {
+        issue(item + kStages - 1);  // into the stage the previous item released
+        cp_async_wait<kStages - 1>();
+        __syncwarp();
+        const int64_t row = item_row(item);
+        const float *xr = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;  // this lane's row
+
+        // approximate keys of this lane's 4*NV experts
+        float kv[NV][4];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+            const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
+            const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
+            kv[m][0] = key_approx(x.x, h.x);
+            kv[m][1] = key_approx(x.y, h.y);
+            kv[m][2] = key_approx(x.z, h.z);
+            kv[m][3] = key_approx(x.w, h.w);
+        }
+        // tau': the K-th largest of the maxima of groups of 8 keys (each
+        // maximum is a key of its own, so tau' is at most the K-th key)
+        constexpr int G = NV / 2;  // groups per lane
+        float gm[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) {
+            const float a = fmaxf(fmaxf(kv[2 * q][0], kv[2 * q][1]), fmaxf(kv[2 * q][2], kv[2 * q][3]));
+            const float b = fmaxf(fmaxf(kv[2 * q + 1][0], kv[2 * q + 1][1]), fmaxf(kv[2 * q + 1][2], kv[2 * q + 1][3]));
+            gm[q] = fmaxf(a, b);
+        }
+        TopValues<P> top;
+        top.init();
+        if constexpr (G <= P) {
+            // all of the lane's group maxima fit the list: sort them (network for 1, 2 or 4)
+            static_assert(G == 1 || G == 2 || G == 4, "groups per lane");
+            auto ce = [](float &hi, float &lo) {
+                const float a = hi, b = lo;
+                hi = fmaxf(a, b);
+                lo = fminf(a, b);
+            };
+            if constexpr (G == 2) ce(gm[0], gm[1]);
+            if constexpr (G == 4) {
+                ce(gm[0], gm[1]);
+                ce(gm[2], gm[3]);
+                ce(gm[0], gm[2]);
+                ce(gm[1], gm[3]);
+                ce(gm[1], gm[2]);
+            }
+#pragma unroll
+            for (int q = 0; q < G; ++q) top.v[q] = gm[q];
+        } else {
+#pragma unroll
+            for (int q = 0; q < G; ++q) top.push(gm[q]);
+        }
+        top.merge_xor(1);
+        top.merge_xor(2);
+        top.merge_xor(4);
+        const float lim = candidate_limit(top.v[K - 1]);
+        unsigned mask = 0;
+#pragma unroll
+        for (int m = 0; m < NV; ++m)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (kv[m][e] >= lim) mask |= 1u << (4 * m + e);
+        if (row >= T) mask = 0;
+
+        // candidate offsets within the row: prefix over the row's 8 lanes
+        const int n = __popc(mask);
+        int incl = n;
+#pragma unroll
+        for (int d = 1; d < kLanesPerRow; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (j >= d) incl += y;
+        }
+        const int excl = incl - n;
+        const int row_n = __shfl_sync(0xffffffffu, incl, lane | (kLanesPerRow - 1));
+
+        if (__all_sync(0xffffffffu, n <= 4 && row_n <= kLanesPerRow)) {
+            // The usual case, without loops: at most 4 candidates per lane and
+            // 8 per row.  Lane j scores the row's j-th candidate and ranks it
+            // against the other 7 through shuffles.
+            unsigned mm = mask;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int p = __ffs(mm) - 1;
+                mm &= mm - 1;
+                if (q < n) cc[excl + q] = 4 * (8 * (p >> 2) + j) + (p & 3);
+            }
+            __syncwarp();
+            const bool has = j < row_n;
+            int c = has ? cc[j] : 0;
+            const float s = sigmoid_rounded_once(xr[c]);
+            const float key = has ? __fadd_rn(s, bias_s[c]) : -INFINITY;
+            c = has ? c : 0x7fffffff;
+            int rank = 0;
+#pragma unroll
+            for (int d = 1; d < kLanesPerRow; ++d) {
+                const int src = (lane & ~(kLanesPerRow - 1)) | ((j + d) & (kLanesPerRow - 1));
+                const float ko = __shfl_sync(0xffffffffu, key, src);
+                const int co = __shfl_sync(0xffffffffu, c, src);
+                rank += (ko > key || (ko == key && co < c)) ? 1 : 0;
+            }
+            if (has && rank < K) {
+                ss[rank] = s;
+                sc[rank] = c;
+            }
+            __syncwarp();
+        } else {
+            const int most = __reduce_max_sync(0xffffffffu, row_n);
+            // rounds of up to kWin candidates per row (one round unless many keys tie)
+            for (int w0 = 0; w0 < most; w0 += kWin) {
+                if (incl > w0 && excl < w0 + kWin) {
+                    unsigned mm = mask;
+                    int off = excl;
+                    while (mm) {
+                        const int p = __ffs(mm) - 1;
+                        mm &= mm - 1;
+                        if (off >= w0 && off < w0 + kWin) cc[off - w0] = 4 * (8 * (p >> 2) + j) + (p & 3);
+                        ++off;
+                    }
+                }
+                __syncwarp();
+                const int wn = min(kWin, row_n - w0);
+                // exact scores: the row's 8 lanes share the round's candidates;
+                // slots [wn, 8) get a sentinel that ranks below everything
+                for (int e = j; e < wn; e += kLanesPerRow) {
+                    const int c = cc[e];
+                    const float s = sigmoid_rounded_once(xr[c]);
+                    cs[e] = s;
+                    ck[e] = __fadd_rn(s, bias_s[c]);
+                }
+                if (j >= wn) {
+                    ck[j] = -INFINITY;
+                    cc[j] = 0x7fffffff;
+                }
+                __syncwarp();
+                // slot of each candidate: its rank under (key desc, index asc)
+                const int dst = w0 == 0 ? 0 : K;
+                for (int e = j; e < wn; e += kLanesPerRow) {
+                    const float ke = ck[e];
+                    const int ce = cc[e];
+                    int rank = 0;
+#pragma unroll
+                    for (int q = 0; q < kLanesPerRow; ++q) {
+                        const float kq = ck[q];
+                        rank += (kq > ke || (kq == ke && cc[q] < ce)) ? 1 : 0;
+                    }
+                    for (int q = kLanesPerRow; q < wn; ++q) {
+                        const float kq = ck[q];
+                        rank += (kq > ke || (kq == ke && cc[q] < ce)) ? 1 : 0;
+                    }
+                    if (rank < K) {
+                        sk[dst + rank] = ke;
+                        ss[dst + rank] = cs[e];
+                        sc[dst + rank] = ce;
+                    }
+                }
+                __syncwarp();
+                if (w0 > 0 && j == 0 && wn > 0) {
+                    // merge this round's best min(K, wn) into the Top-K so far
+                    float mk[K], ms[K];
+                    int mc[K];
+                    const int nb = min(K, wn);
+                    int a = 0, b = 0;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        const bool take_b =
+                            b < nb && (sk[K + b] > sk[a] || (sk[K + b] == sk[a] && sc[K + b] < sc[a]));
+                        const int src = take_b ? K + b : a;
+                        mk[k] = sk[src];
+                        ms[k] = ss[src];
+                        mc[k] = sc[src];
+                        b += take_b ? 1 : 0;
+                        a += take_b ? 0 : 1;
+                    }
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        sk[k] = mk[k];
+                        ss[k] = ms[k];
+                        sc[k] = mc[k];
+                    }
+                }
+                __syncwarp();
+            }
+        }
+
+        // gates (fp64, slot order), outputs, histogram: lane j writes slot j
+        if (row < T && j < K) {
+            double sum = 0.0;
+#pragma unroll
+            for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)ss[k]);
+            const int c = sc[j];
+            topk_idx[row * K + j] = c;
+            gates[row * K + j] = __double2float_rn(__ddiv_rn((double)ss[j], sum));
+            if ((unsigned)c < (unsigned)Nr) atomicAdd(&hist[c], 1);
+        }
+        __syncwarp();  // the ring stage and the candidate slots are reused
+
+        if (want_tiles && (item & 7) == 7) {
+            const int tile = (int)blockIdx.x + (item >> 3) * (int)gridDim.x;
+            __syncthreads();
+            for (int e = threadIdx.x; e < Nr; e += kThreads) {
+                const int v = hist_tile[e];
+                tile_counts[(size_t)tile * Nr + e] = v;
+                hist_total[e] += v;
+                hist_tile[e] = 0;
+            }
+            __syncthreads();
+        }
+    }
+    cp_async_wait<0>();  // the zero-fill copies issued past the last item
+    __syncthreads();
+    for (int e = threadIdx.x; e < Nr; e += kThreads)
+        if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
+}
+
+// max over i of |approximate score - exact score| as the bits of a
+// non-negative float (those order like unsigned integers)
+__global__ void score_error_kernel(const float *__restrict__ x, int64_t n, unsigned *__restrict__ max_bits) {
+    float worst = 0.0f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        worst = fmaxf(worst, fabsf(key_approx(x[i], 0.5f) - sigmoid_rounded_once(x[i])));
+    atomicMax(max_bits, __float_as_uint(worst));
+}
+
+}  // namespace
+
+namespace {
+
+// Per (kernel, device): the dynamic shared-memory grant is set once and the
+// resident CTAs per SM are measured once (the persistent grid's size).
+struct VecSetup {
+    const void *kern;
+    int device;
+    int blocks_per_sm;
+};
+std::mutex g_vec_mu;
+VecSetup g_vec[64];
+int g_num_vec = 0;
+
+cudaError_t vec_setup(const void *kern, size_t smem, int *blocks_per_sm) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(g_vec_mu);
+    for (int i = 0; i < g_num_vec; ++i)
+        if (g_vec[i].kern == kern && g_vec[i].device == dev) {
+            *blocks_per_sm = g_vec[i].blocks_per_sm;
+            return cudaSuccess;
+        }
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int b = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (b < 1) b = 1;
+    if (g_num_vec < 64) g_vec[g_num_vec++] = {kern, dev, b};
+    *blocks_per_sm = b;
+    return cudaSuccess;
+}
+
+template <int K, int NV>
+cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, int32_t *topk_idx, float *gates,
+                       int32_t *counts, int32_t *tile_counts, int num_sms, cudaStream_t stream) {
+    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV>);
+    const size_t smem = vec_ring_bytes<NV>();
+    int per_sm = 1;
+    cudaError_t err = vec_setup(kern, smem, &per_sm);
+    if (err != cudaSuccess) return err;
+    const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    int grid = num_sms * per_sm;
+    if (grid > num_tiles) grid = num_tiles;
+    router_logits_vec_kernel<K, NV><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates, counts,
+                                                                      tile_counts);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
                                  float *gates, int32_t *counts, int32_t *tile_counts, int num_sms,
                                  cudaStream_t stream) {
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
+    if (Nr % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
+        // vector kernel: persistent CTAs, as many per SM as fit
+        const int nv = Nr <= 64 ? 2 : (Nr <= 128 ? 4 : 8);
+        switch (K * 16 + nv) {
+#define EBL_VCASE(KK, NN) \
+    case KK * 16 + NN:    \
+        return launch_vec<KK, NN>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream);
+#define EBL_VCASES(KK) EBL_VCASE(KK, 2) EBL_VCASE(KK, 4) EBL_VCASE(KK, 8)
+            EBL_VCASES(1)
+            EBL_VCASES(2)
+            EBL_VCASES(3)
+            EBL_VCASES(4)
+            EBL_VCASES(5)
+            EBL_VCASES(6)
+            EBL_VCASES(7)
+            EBL_VCASES(8)
+#undef EBL_VCASES
+#undef EBL_VCASE
+            default:
+                return cudaErrorInvalidValue;
+        }
+    }
+    // row kernel: any N_r and alignment
     int grid = num_sms * 16;
     if (grid > num_tiles) grid = num_tiles;
     switch (K) {
@@ -213,5 +678,17 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
     }
     return cudaGetLastError();
 }
+
+cudaError_t launch_score_error(const float *x, int64_t n, float *max_err, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(max_err, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    score_error_kernel<<<(int)blocks, 256, 0, stream>>>(x, n, reinterpret_cast<unsigned *>(max_err));
+    return cudaGetLastError();
+}
+
+float logits_key_error_bound() { return kKeyErr; }
 
 }  // namespace ebl

@@ -1,7 +1,13 @@
-// selftest.cu -- checks the bounded pipeline wait that every kernel here uses:
-// one thread waits, with a short limit, on an mbarrier that nothing arrives
-// on.  The wait must give up, the kernel must report EBL_ST_TIMEOUT in the
-// status word and return, and the CUDA context must stay usable.
+// selftest.cu -- self-tests of two device-side assumptions.
+//
+// ebl_selftest_wait_timeout: the bounded pipeline wait that every kernel here
+// uses.  One thread waits, with a short limit, on an mbarrier that nothing
+// arrives on; the wait must give up, the kernel must report EBL_ST_TIMEOUT in
+// the status word and return, and the CUDA context must stay usable.
+//
+// ebl_selftest_score_error: the distance between the approximate score the
+// logits-mode ranking uses and the exact one, against the bound that ranking
+// assumes.
 
 #include "../../include/ebl.h"
 #include "launch.h"
@@ -30,5 +36,15 @@ extern "C" int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us,
     if (limit_us < 1 || limit_us > 1000000) return EBL_EINVAL;
     ebl::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status, 1000ull * limit_us);
     if (cudaGetLastError() != cudaSuccess) return EBL_ECUDA;
+    return EBL_OK;
+}
+
+extern "C" int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound,
+                                        ebl_stream_t stream) {
+    if (n < 0 || !max_err || (reinterpret_cast<uintptr_t>(max_err) & 3u)) return EBL_EINVAL;
+    if (n > 0 && (!x || (reinterpret_cast<uintptr_t>(x) & 3u))) return EBL_EINVAL;
+    if (bound) *bound = ebl::logits_key_error_bound();
+    if (ebl::launch_score_error(x, n, max_err, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return EBL_ECUDA;
     return EBL_OK;
 }

@@ -143,9 +143,11 @@ int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const
  * formulas exactly (up to a last-ulp difference between two fp64 exp
  * implementations, about one value in 2^28).
  *
- * logits  device, fp32 [T, N_r].
+ * logits  device, fp32 [T, N_r], 4-byte aligned.  With N_r % 4 == 0 and a
+ *         16-byte aligned base the logits are read from HBM once; otherwise
+ *         a slower kernel reads them twice (same results).
  * N_r     1 <= N_r <= 256 (any value).  K: 1 <= K <= min(8, N_r).
- * Other arguments as router_forward.
+ * Other arguments as router_forward.  Logits and bias are assumed finite.
  */
 int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K,
                           int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
@@ -286,6 +288,19 @@ int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *d
  * timeout path is exercised without faulting or hanging a GPU.
  */
 int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us, ebl_stream_t stream);
+
+/*
+ * ebl_selftest_score_error -- checks the approximation router_forward_logits
+ * ranks with.  That mode scores every expert with an approximate sigmoid
+ * (0.5 + 0.5 tanh(x/2), one tanh.approx.f32) and evaluates the exact score
+ * only for experts whose approximate key is within a bound of the K-th
+ * largest; the bound must exceed the approximation's error.  This call writes
+ *   *max_err = max_i | approx(x_i) - (float)(1 / (1 + exp(-(double)x_i))) |
+ * (device fp32, 4-byte aligned) and, if bound is not NULL, the absolute error
+ * bound the ranking assumes to *bound (host).  x: device fp32 [n], n >= 0.
+ * No counterpart on the pages: it tests an implementation assumption.
+ */
+int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound, ebl_stream_t stream);
 
 /*
  * ebl_read_internal_status -- copy the library-owned status word (used when a

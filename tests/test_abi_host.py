@@ -90,6 +90,9 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine(FAKE, FAKE, FAKE, 100, 64, 9, FAKE, None, None) == EINVAL
     assert lib.moe_combine(FAKE, FAKE, FAKE, 0, 64, 2, FAKE, None, None) == 0
     assert lib.ebl_read_internal_status(None, 0) == EINVAL
+    assert lib.ebl_selftest_score_error(FAKE, -1, FAKE, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(FAKE, 10, None, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(None, 10, FAKE, None, None) == EINVAL
 
 
 def test_binding_has_no_cpu_fallback():

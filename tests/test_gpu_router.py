@@ -11,10 +11,18 @@ from tests.parity import STATE_RTOL, assert_gemm_parity, rel_err, tile_hist, to_
 pytestmark = pytest.mark.gpu
 
 
-def _run_logits(logits, bias, K, want_tiles=True):
+def _run_logits(logits, bias, K, want_tiles=True, misalign=False):
+    """misalign: place the logits 4 bytes past a 16-byte boundary, which sends
+    them through the row kernel instead of the vector kernel."""
     dev = torch.device("cuda:0")
     T, Nr = logits.shape
-    x = logits.to(dev)
+    if misalign:
+        buf = torch.empty(T * Nr + 1, dtype=torch.float32, device=dev)
+        buf[1:] = logits.reshape(-1).to(dev)
+        x = buf[1:].view(T, Nr)
+        assert x.data_ptr() % 16 == 4
+    else:
+        x = logits.to(dev)
     b = bias.to(dev)
     counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
     tiles = torch.full(((T + 127) // 128, Nr), -7, dtype=torch.int32, device=dev) if want_tiles else None
@@ -37,8 +45,9 @@ LOGITS_CASES = [
 ]
 
 
+@pytest.mark.parametrize("misalign", [False, True])
 @pytest.mark.parametrize("T,Nr,K,quant,bk", LOGITS_CASES)
-def test_logits_mode_bit_exact(cuda_device, T, Nr, K, quant, bk):
+def test_logits_mode_bit_exact(cuda_device, T, Nr, K, quant, bk, misalign):
     logits = synth.logits_normal(T, Nr, seed=100 + T + Nr + K, quant8=quant)
     if bk == "small":
         bias = torch.randn(Nr, generator=torch.Generator().manual_seed(K)) * 0.01
@@ -46,7 +55,7 @@ def test_logits_mode_bit_exact(cuda_device, T, Nr, K, quant, bk):
         bias = (torch.randint(-2, 3, (Nr,), generator=torch.Generator().manual_seed(K)) * 0.125).float()
     else:
         bias = synth.dead_start_bias(Nr, n_dead=min(8, Nr - K))
-    idx, gates, counts, tiles = _run_logits(logits, bias, K)
+    idx, gates, counts, tiles = _run_logits(logits, bias, K, misalign=misalign)
     ref = oracle.router_logits(logits.numpy(), bias.numpy(), K, tile_tokens=128)
     assert np.array_equal(idx, ref.idx)
     assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
@@ -199,3 +208,46 @@ def test_logits_mode_all_equal_keys(cuda_device):
     assert np.all(gates == np.float32(0.25))
     ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
     assert np.array_equal(idx, ref.idx) and np.array_equal(counts, ref.counts)
+
+
+@pytest.mark.parametrize("misalign", [False, True])
+@pytest.mark.parametrize("Nr,K", [(256, 4), (128, 8), (64, 3), (256, 1)])
+def test_logits_mode_many_tied_candidates(cuda_device, Nr, K, misalign):
+    """Rows where 1..90 experts tie at the top key (logits on a 1/8 grid, bias
+    on a 1/8 grid for half of the rows): the candidates of a row are scored in
+    one to three rounds of 32 and merged, and equal keys go to the lower
+    index."""
+    T = 3000
+    g = torch.Generator().manual_seed(Nr * 10 + K)
+    x = torch.round(torch.randn(T, Nr, generator=g) * 8) / 8 - 4.0
+    ties = torch.randint(1, min(90, Nr) + 1, (T,), generator=g)
+    for t in range(T):
+        cols = torch.randperm(Nr, generator=g)[: int(ties[t])]
+        x[t, cols] = 1.5
+    bias = torch.zeros(Nr)
+    bias[torch.randperm(Nr, generator=g)[: Nr // 4]] = -0.125
+    idx, gates, counts, tiles = _run_logits(x, bias, K, misalign=misalign)
+    ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx)
+    assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
+    assert np.array_equal(counts, ref.counts)
+    assert np.array_equal(tiles, ref.tile_counts)
+
+
+def test_logits_score_error_within_bound(cuda_device):
+    """The approximate score logits mode ranks with stays well inside the
+    error bound its candidate limit assumes, over a dense sweep of [-40, 40],
+    the values near 0, and random finite fp32 bit patterns."""
+    dev = cuda_device
+    sweep = torch.linspace(-40.0, 40.0, 1 << 24, device=dev)
+    tiny = torch.linspace(-1e-3, 1e-3, 1 << 20, device=dev)
+    bits = torch.randint(0, 1 << 31, (1 << 22,), generator=torch.Generator().manual_seed(3), dtype=torch.int64)
+    bits = bits.to(torch.int32).view(torch.float32)
+    rnd = bits[torch.isfinite(bits)].to(dev)
+    rnd = torch.cat([rnd, -rnd])
+    for x in (sweep, tiny, rnd):
+        err, bound = ebl.selftest_score_error(x.contiguous())
+        assert 0.0 < bound <= 2.0 ** -8
+        assert err * 4.0 <= bound, (err, bound)
+    err, _ = ebl.selftest_score_error(torch.tensor([0.0, 1.0, -1.0], device=dev))
+    assert err < 2.0 ** -11
