@@ -42,6 +42,10 @@ LOGITS_CASES = [
     (129, 200, 5, True, "ties"),
     (1, 33, 2, False, "small"),
     (127, 256, 7, False, "dead"),
+    (777, 4, 2, True, "ties"),           # the smallest row the vector kernel takes (one float4)
+    (500, 68, 6, False, "small"),        # just past 64 experts: 4 float4 per lane, 3 of them partly padding
+    (500, 132, 3, True, "dead"),         # just past 128: 8 float4 per lane
+    (600, 252, 8, True, "ties"),         # ragged last column block
 ]
 
 
@@ -251,3 +255,29 @@ def test_logits_score_error_within_bound(cuda_device):
         assert err * 4.0 <= bound, (err, bound)
     err, _ = ebl.selftest_score_error(torch.tensor([0.0, 1.0, -1.0], device=dev))
     assert err < 2.0 ** -11
+
+
+@pytest.mark.parametrize("misalign", [False, True])
+def test_logits_mode_saturated_scores(cuda_device, misalign):
+    """Logits of scale 60: most sigmoids round to exactly 0.0 or 1.0 in fp32,
+    so dozens of experts per row share the top key and the lowest indices
+    must win; a small bias on a 1/64 grid splits some of them."""
+    T, Nr, K = 2000, 256, 4
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(T, Nr, generator=g) * 60.0
+    bias = (torch.randint(-1, 2, (Nr,), generator=g) / 64.0).float()
+    idx, gates, counts, tiles = _run_logits(x, bias, K, misalign=misalign)
+    ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx)
+    assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
+    assert np.array_equal(counts, ref.counts)
+    assert np.array_equal(tiles, ref.tile_counts)
+
+
+def test_microbench_runs_every_entry_point(cuda_device, capsys):
+    from expert_bias_load_b200 import microbench
+    for op in ("router", "zloss", "logits", "smebu", "sign", "dispatch", "combine"):
+        microbench.main([op, "--tokens", "4096", "--hidden", "256", "--experts", "64", "--topk", "4",
+                         "--warmup", "1", "--reps", "2"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if " ms, " in l]
+    assert len(lines) == 7
