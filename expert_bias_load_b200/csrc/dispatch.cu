@@ -12,12 +12,15 @@
 //   3. seg_scan    one CTA: expert totals, offsets (exclusive scan over
 //                  experts), segment bases (exclusive scan over segments)
 //   4. tile_bases  per tile, per expert base = segment base + earlier tiles
-// and the copy kernel ranks each tile's pairs in pair order from its tile base
-// (warp match on expert ids, 32 pairs at a time) and streams every hidden row
-// once from HBM to its K destinations with 16-byte loads and stores.
+// then rank_kernel ranks each tile's pairs in pair order from its tile base
+// (warp match on expert ids, 32 pairs at a time) into dest and perm, and
+// copy_kernel streams every hidden row once from HBM to its K destinations
+// with TMA bulk copies through a shared-memory ring.
 //
 // Combine: out[t,:] = sum_k g[t,k] * Y[dest[t*K+k],:], one warp per token,
 // fp32 fma chain in slot order from 0 (deterministic, no atomics).
+
+#include <mutex>
 
 #include "launch.h"
 #include "ptx.cuh"
@@ -26,8 +29,6 @@ namespace ebl {
 namespace {
 
 constexpr int kSegTiles = 32;
-constexpr int kCopyThreads = 256;
-constexpr int kCopyWarps = kCopyThreads / 32;
 
 __host__ __device__ inline int num_tiles_of(int T) { return (T + kTileTokens - 1) / kTileTokens; }
 __host__ __device__ inline int num_segs_of(int tiles) { return (tiles + kSegTiles - 1) / kSegTiles; }
@@ -119,83 +120,166 @@ __global__ void __launch_bounds__(kMaxExperts) tile_bases_kernel(const int32_t *
     }
 }
 
-__global__ void __launch_bounds__(kCopyThreads) rank_copy_kernel(const uint4 *__restrict__ hidden,
-                                                                 const int32_t *__restrict__ topk_idx,
-                                                                 const int32_t *__restrict__ bases, int T,
-                                                                 int d8, int Nr, int K, int32_t *__restrict__ perm,
-                                                                 int32_t *__restrict__ dest,
-                                                                 uint4 *__restrict__ dispatched,
-                                                                 int32_t *__restrict__ status) {
-    __shared__ int cnt[kMaxExperts];
-    __shared__ int dst_s[kTileTokens * kMaxTopK];
+// Rank: one warp per tile ranks the tile's pairs in pair order from the tile's
+// bases, 32 pairs at a time (warp match on the expert ids), and writes dest
+// and perm.  Expert ids outside [0, N_r) get dest = -1; so do pairs whose
+// rank falls outside [0, T*K), which only tile counts that disagree with
+// topk_idx can cause.  Both raise EBL_ST_BAD_EXPERT.
+constexpr int kRankWarps = 4;
+
+__global__ void __launch_bounds__(kRankWarps * 32) rank_kernel(const int32_t *__restrict__ topk_idx,
+                                                               const int32_t *__restrict__ bases, int T, int Nr,
+                                                               int K, int32_t *__restrict__ perm,
+                                                               int32_t *__restrict__ dest,
+                                                               int32_t *__restrict__ status) {
+    __shared__ int cnt_s[kRankWarps][kMaxExperts];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_tiles = num_tiles_of(T);
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int row0 = tile * kTileTokens;
-        const int rows = min(kTileTokens, T - row0);
-        const int np = rows * K;
-        const size_t p0 = (size_t)row0 * K;
-        for (int e = threadIdx.x; e < Nr; e += kCopyThreads) cnt[e] = bases[(size_t)tile * Nr + e];
-        for (int q = threadIdx.x; q < np; q += kCopyThreads) dst_s[q] = topk_idx[p0 + q];
-        __syncthreads();
-        if (warp == 0) {
-            const long long num_rows = (long long)T * K;
-            bool bad = false, bad_base = false;
-            for (int q0 = 0; q0 < np; q0 += 32) {
-                const int q = q0 + lane;
-                const bool valid = q < np;
-                int e = valid ? dst_s[q] : -1;
-                const bool good = valid && (unsigned)e < (unsigned)Nr;
-                if (valid && !good) bad = true;
-                if (!good) e = -1 - (valid ? 0 : 1);  // invalid lanes never match good ones
-                const uint32_t peers = __match_any_sync(0xffffffffu, e);
-                int j = -1;
-                if (good) j = cnt[e] + __popc(peers & lanemask_lt());
-                __syncwarp();
-                if (good && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
-                if (good && (unsigned)j >= (unsigned)num_rows) {  // tile counts that disagree with topk_idx
-                    bad_base = true;
-                    j = -1;
-                }
-                if (valid) {
-                    dst_s[q] = j;
-                    dest[p0 + q] = j;
-                    if (j >= 0) perm[j] = (row0 + q / K);
-                }
-                __syncwarp();
-            }
-            if (bad || bad_base) atomicOr(status, kStBadExpert);
+    const int tile = blockIdx.x * kRankWarps + warp;
+    if (tile >= num_tiles_of(T)) return;  // whole warps only; no CTA barrier below
+    int *cnt = cnt_s[warp];
+    for (int e = lane; e < Nr; e += 32) cnt[e] = bases[(size_t)tile * Nr + e];
+    __syncwarp();
+    const int row0 = tile * kTileTokens;
+    const int np = min(kTileTokens, T - row0) * K;
+    const size_t p0 = (size_t)row0 * K;
+    const long long num_pairs = (long long)T * K;
+    bool bad = false;
+    for (int q0 = 0; q0 < np; q0 += 32) {
+        const int q = q0 + lane;
+        const bool valid = q < np;
+        int e = valid ? topk_idx[p0 + q] : -1;
+        const bool good = valid && (unsigned)e < (unsigned)Nr;
+        if (valid && !good) bad = true;
+        if (!good) e = valid ? -1 : -2;  // never equal to a good id
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        int j = -1;
+        if (good) j = cnt[e] + __popc(peers & lanemask_lt());
+        __syncwarp();
+        if (good && lane == __ffs(peers) - 1) cnt[e] += __popc(peers);
+        __syncwarp();
+        if (good && (unsigned long long)j >= (unsigned long long)num_pairs) {
+            bad = true;
+            j = -1;
         }
-        __syncthreads();
-        // stream the rows: warp w copies rows w, w + 8, ...
-        for (int r = warp; r < rows; r += kCopyWarps) {
-            const uint4 *src = hidden + (size_t)(row0 + r) * d8;
-            int dj[kMaxTopK];
-#pragma unroll
-            for (int k = 0; k < kMaxTopK; ++k) dj[k] = k < K ? dst_s[r * K + k] : -1;
-            int c = lane;
-            for (; c + 96 < d8; c += 128) {
-                const uint4 v0 = __ldcs(src + c), v1 = __ldcs(src + c + 32), v2 = __ldcs(src + c + 64),
-                            v3 = __ldcs(src + c + 96);
-#pragma unroll
-                for (int k = 0; k < kMaxTopK; ++k) {
-                    if (dj[k] < 0) continue;
-                    uint4 *dst = dispatched + (size_t)dj[k] * d8;
-                    __stcs(dst + c, v0);
-                    __stcs(dst + c + 32, v1);
-                    __stcs(dst + c + 64, v2);
-                    __stcs(dst + c + 96, v3);
-                }
-            }
-            for (; c < d8; c += 32) {
-                const uint4 v = __ldcs(src + c);
-#pragma unroll
-                for (int k = 0; k < kMaxTopK; ++k)
-                    if (dj[k] >= 0) __stcs(dispatched + (size_t)dj[k] * d8 + c, v);
-            }
+        if (valid) {
+            dest[p0 + q] = j;
+            if (j >= 0) perm[j] = row0 + q / K;
         }
-        __syncthreads();
     }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, kStBadExpert);
+}
+
+// Copy: TMA bulk copies.  One warp per CTA; lane 0 streams the CTA's rows
+// (a contiguous block of tokens) through a ring of shared-memory stages in
+// chunks of up to kChunkBytes: one bulk load per chunk, then one bulk store
+// per destination row.  kCopyAhead loads are in flight; a stage is refilled
+// only after the stores issued kCopyAhead chunks earlier have read it.  The
+// lanes hold the dest entries of 32 rows at a time, loaded one batch ahead.
+constexpr int kCopyStages = 12;
+constexpr int kCopyAhead = kCopyStages / 2;
+constexpr int kChunkBytes = 8192;
+constexpr size_t kCopySmemBytes = (size_t)kCopyStages * kChunkBytes;
+
+__device__ __forceinline__ void bulk_load(void *smem, const void *gmem, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem)),
+                 "l"(gmem), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_store(void *gmem, const void *smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem), "r"(smem_u32(smem)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(32) copy_kernel(const uint8_t *__restrict__ hidden, const int32_t *__restrict__ dest,
+                                                  int T, int row_bytes, int K, uint8_t *__restrict__ dispatched,
+                                                  int32_t *__restrict__ status) {
+    extern __shared__ __align__(128) uint8_t ring[];  // kCopyStages x kChunkBytes
+    __shared__ uint64_t full[kCopyStages];
+    __shared__ int abort_flag;
+    const int lane = threadIdx.x;
+    const int64_t per = ((int64_t)T + gridDim.x - 1) / gridDim.x;
+    const int64_t r0 = (int64_t)blockIdx.x * per;
+    const int64_t r1 = min((int64_t)T, r0 + per);
+    if (r0 >= r1) return;
+    if (lane == 0) {
+        for (int s = 0; s < kCopyStages; ++s) mbar_init(&full[s], 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const int cpr = (row_bytes + kChunkBytes - 1) / kChunkBytes;  // chunks per row
+    const int64_t U = (r1 - r0) * cpr;
+    auto chunk_row = [&](int64_t u) { return r0 + u / cpr; };
+    auto chunk_off = [&](int64_t u) { return (int)(u % cpr) * kChunkBytes; };
+    auto chunk_bytes = [&](int64_t u) { return (uint32_t)min(kChunkBytes, row_bytes - chunk_off(u)); };
+    auto issue_load = [&](int64_t v) {
+        const int s = (int)(v % kCopyStages);
+        const uint32_t nb = chunk_bytes(v);
+        mbar_arrive_expect_tx(&full[s], nb);
+        bulk_load(ring + (size_t)s * kChunkBytes, hidden + chunk_row(v) * row_bytes + chunk_off(v), nb, &full[s]);
+    };
+    auto load_dest = [&](int64_t row, int (&dk)[kMaxTopK]) {
+#pragma unroll
+        for (int k = 0; k < kMaxTopK; ++k) dk[k] = (k < K && row < r1) ? dest[row * K + k] : -1;
+    };
+
+    if (lane == 0)
+        for (int64_t v = 0; v < min((int64_t)kCopyAhead, U); ++v) issue_load(v);
+    int64_t batch0 = r0;  // lane l holds the dest entries of row batch0 + l in dk
+    int dk[kMaxTopK], dn[kMaxTopK];
+    load_dest(batch0 + lane, dk);
+    load_dest(batch0 + 32 + lane, dn);
+    int64_t u = 0;
+    for (; u < U; ++u) {
+        const int64_t row = chunk_row(u);
+        if (row >= batch0 + 32) {  // next batch of 32 rows (warp-uniform)
+            batch0 += 32;
+#pragma unroll
+            for (int k = 0; k < kMaxTopK; ++k) dk[k] = dn[k];
+            load_dest(batch0 + 32 + lane, dn);
+        }
+        const int s = (int)(u % kCopyStages);
+        int ok = 1;
+        if (lane == 0) {
+            const int64_t v = u + kCopyAhead;
+            if (v < U) {
+                bulk_wait_read<kCopyAhead - 1>();
+                issue_load(v);
+            }
+            ok = mbar_wait(&full[s], (uint32_t)((u / kCopyStages) & 1), &abort_flag) ? 1 : 0;
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        const int src = (int)(row - batch0);
+        const int off = chunk_off(u);
+        const uint32_t nb = chunk_bytes(u);
+#pragma unroll
+        for (int k = 0; k < kMaxTopK; ++k) {
+            const int j = __shfl_sync(0xffffffffu, dk[k], src);
+            if (lane == 0 && k < K && j >= 0)
+                bulk_store(dispatched + (int64_t)j * row_bytes + off, ring + (size_t)s * kChunkBytes, nb);
+        }
+        if (lane == 0) bulk_commit();
+    }
+    if (lane == 0) {
+        if (u < U) {
+            // a load never landed: report, then give the loads already issued a
+            // bounded time to land before the shared memory goes away
+            atomicOr(status, kStTimeout);
+            const int64_t issued = min(U, u + kCopyAhead);
+            for (int64_t w = u; w < issued; ++w)
+                mbar_wait(&full[w % kCopyStages], (uint32_t)((w / kCopyStages) & 1), &abort_flag, 100000000ull);
+        }
+        bulk_wait_all();  // the stores read shared memory until they complete
+    }
+    __syncwarp();
 }
 
 __device__ __forceinline__ void fma_bf16x8(const uint4 v, float g, float (&acc)[8]) {
@@ -246,6 +330,27 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4 *__restrict__ 
 
 }  // namespace
 
+namespace {
+
+// The copy kernel's dynamic shared-memory grant, set once per device.
+std::mutex g_copy_mu;
+bool g_copy_ready[64] = {};
+
+cudaError_t copy_setup() {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(g_copy_mu);
+    if (dev >= 0 && dev < 64 && g_copy_ready[dev]) return cudaSuccess;
+    err = cudaFuncSetAttribute(reinterpret_cast<const void *>(&copy_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCopySmemBytes);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64) g_copy_ready[dev] = true;
+    return cudaSuccess;
+}
+
+}  // namespace
+
 size_t dispatch_workspace_bytes(int T, int Nr) {
     const int tiles = num_tiles_of(T);
     const int segs = num_segs_of(tiles);
@@ -268,11 +373,14 @@ cudaError_t launch_dispatch(const uint16_t *hidden, const int32_t *topk_idx, con
     seg_sums_kernel<<<segs, kMaxExperts, 0, stream>>>(tc, tiles, Nr, ws_seg);
     seg_scan_kernel<<<1, kMaxExperts, 0, stream>>>(ws_seg, segs, Nr, (long long)T * K, offsets, status);
     tile_bases_kernel<<<segs, kMaxExperts, 0, stream>>>(tc, ws_seg, tiles, Nr, ws_tiles);
-    int grid = num_sms * 4;
-    if (grid > tiles) grid = tiles;
-    rank_copy_kernel<<<grid, kCopyThreads, 0, stream>>>(reinterpret_cast<const uint4 *>(hidden), topk_idx,
-                                                        ws_tiles, T, d / 8, Nr, K, perm, dest,
-                                                        reinterpret_cast<uint4 *>(dispatched), status);
+    rank_kernel<<<(tiles + kRankWarps - 1) / kRankWarps, kRankWarps * 32, 0, stream>>>(topk_idx, ws_tiles, T, Nr, K,
+                                                                                      perm, dest, status);
+    cudaError_t err = copy_setup();
+    if (err != cudaSuccess) return err;
+    int grid = num_sms * 2;  // two 96 KB rings per SM
+    if (grid > T) grid = T;
+    copy_kernel<<<grid, 32, kCopySmemBytes, stream>>>(reinterpret_cast<const uint8_t *>(hidden), dest, T, d * 2, K,
+                                                      reinterpret_cast<uint8_t *>(dispatched), status);
     return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@ CASES = [
     (127, 24, 16, 3, False),
     (5000, 136, 64, 2, True),
     (3000, 1024, 128, 8, False),
+    (700, 8256, 32, 2, False),           # rows of 16.5 KB: copied in 8 KB + 8 KB + 128 B pieces
 ]
 
 
