@@ -287,16 +287,23 @@ def main():
     flops = 2.0 * T * d * Nr
     alg_bytes = 2.0 * T * d + 8.0 * T * K + 2.0 * Nr * d + 8.0 * Nr
     achieved = flops / (router_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic("ties_full"),
+    # The router is timed back to back for total_ms; a loop of a second or more
+    # runs under the power cap like the sustained GEMM measurement, a shorter
+    # one like the burst measurement.
+    sustained = peaks.get("bf16_tflops_sustained")
+    long_loop = total_ms >= 1000.0 and sustained
+    peak = sustained if long_loop else peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic("ties_full"),
                 "kernel": "router_gemm_kernel<4>", "kernel_ms": router_ms,
-                "peak_source": "%s burst bf16 (MEASURED_PEAKS.json)" % peaks["source"],
-                "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                      if peaks.get("bf16_tflops_sustained") else None),
+                "peak_source": "%s %s bf16 (MEASURED_PEAKS.json); timed loop %.2f s" % (
+                    peaks["source"], "sustained" if long_loop else "burst", total_ms / 1e3),
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / sustained if sustained else None,
                 "hbm_view": {"alg_bytes": alg_bytes, "achieved_gbs": alg_bytes / (router_ms / 1e3) / 1e9,
                              "peak_gbs": peaks["hbm_gbs"],
                              "frac": alg_bytes / (router_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
-                "roofline_time_ms": max(flops / peaks["bf16_tflops"] / 1e12, alg_bytes / peaks["hbm_gbs"] / 1e9) * 1e3}
+                "roofline_time_ms": max(flops / peak / 1e12, alg_bytes / peaks["hbm_gbs"] / 1e9) * 1e3}
     roofline["frac_of_roofline_step"] = roofline["roofline_time_ms"] / ms_step
 
     # ---- end to end through the public API with host buffers
