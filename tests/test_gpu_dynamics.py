@@ -128,3 +128,56 @@ def test_router_step_in_cuda_graph(cuda_device):
         state[mode] = (b.clone(), m.clone(), idx.clone(), g.clone())
     for a, c in zip(state["eager"], state["graph"]):
         assert torch.equal(a, c)
+
+
+def test_full_step_in_cuda_graph(cuda_device):
+    """Router with tile counts, SMEBU, dispatch and combine captured once in a
+    CUDA graph: replays give the same bias, indices, dispatched rows and
+    combined output as eager launches (the TMA copy and the scan kernels
+    included)."""
+    dev = cuda_device
+    T, d, Nr, K = 3000, 512, 128, 4
+    W = synth.router_weight(Nr, d, seed=21).to(dev)
+    h = synth.hidden_normal(T, d, seed=22, device=dev)
+    tiles_n = (T + 127) // 128
+    state = {}
+    for mode in ("eager", "graph"):
+        b = synth.dead_start_bias(Nr, device=dev)
+        m = torch.zeros(Nr, device=dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        g = torch.empty(T, K, device=dev)
+        tiles = torch.empty(tiles_n, Nr, dtype=torch.int32, device=dev)
+        offsets = torch.empty(Nr + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * K, dtype=torch.int32, device=dev)
+        dest = torch.empty(T * K, dtype=torch.int32, device=dev)
+        X = torch.empty(T * K, d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, ebl.dispatch_workspace_bytes(T, Nr)), dtype=torch.uint8, device=dev)
+        out = torch.empty(T, d, device=dev)
+
+        def step(stream=None):
+            ebl.router_forward(h, W, b, K, counts, topk_idx=idx, gates=g, tile_counts=tiles, stream=stream)
+            ebl.smebu_step(counts, b, m, reset_counts=True, stream=stream)
+            ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles, offsets=offsets, perm=perm, dest=dest, dispatched=X,
+                             workspace=ws, stream=stream)
+            ebl.moe_combine(X, g, dest, out=out, stream=stream)
+
+        if mode == "eager":
+            for _ in range(3):
+                step()
+        else:
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                step(s)                               # first calls set up the kernels outside the graph
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(torch.cuda.current_stream())
+            for _ in range(2):
+                graph.replay()
+        torch.cuda.synchronize()
+        state[mode] = (b.clone(), m.clone(), idx.clone(), dest.clone(), X.clone(), out.clone())
+    for a, c in zip(state["eager"], state["graph"]):
+        assert torch.equal(a, c)
