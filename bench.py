@@ -249,6 +249,14 @@ def main():
 
     dp_step = DataParallelRouterStep(route, update)  # all-reduces the loads when world > 1
 
+    def max_over_ranks(vals):
+        """Element-wise max of per-rank timings (every rank calls this at the same point)."""
+        if world == 1:
+            return list(vals)
+        t = torch.tensor(vals, device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return [float(x) for x in t]
+
     def step(ev0=None, ev1=None):
         rec[0], rec[1] = ev0, ev1
         dp_step(h, bias, mom, counts, maxvio)
@@ -385,7 +393,7 @@ def main():
             tr += ev[0].elapsed_time(ev[1])
             td += ev[1].elapsed_time(ev[2])
             tc += ev[2].elapsed_time(ev[3])
-        tr, td, tc = tr / reps, td / reps, tc / reps
+        tr, td, tc = max_over_ranks([tr / reps, td / reps, tc / reps])
         disp_bytes = T * d * 2 + T * K * d * 2
         comb_bytes = T * K * d * 2 + T * d * 4
         full = {"metric": "tokens/s through router+SMEBU+dispatch+identity expert+combine",
@@ -410,7 +418,7 @@ def main():
             ebl.router_forward_zloss(h, W, bias, K, counts, zl, topk_idx=idx, gates=gates, stream=stream)
         ev[1].record(stream)
         torch.cuda.synchronize()
-        extra["zloss_router_ms"] = ev[0].elapsed_time(ev[1]) / reps
+        extra["zloss_router_ms"] = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
         del zl
         x = synth.logits_normal(T, Nr, seed=synth.step_seed(WORKLOAD, 1) + 1000 * rank, device=dev, quant8=True)
         for _ in range(2):
@@ -421,7 +429,7 @@ def main():
             ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=gates, stream=stream)
         ev[1].record(stream)
         torch.cuda.synchronize()
-        lm = ev[0].elapsed_time(ev[1]) / reps
+        lm = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
         lbytes = T * Nr * 4 + T * K * 8
         extra["logits_mode"] = {"tokens_per_s": T * world / (lm / 1e3), "ms": lm,
                                 "achieved_gbs": lbytes / (lm / 1e3) / 1e9,
