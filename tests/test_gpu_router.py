@@ -103,6 +103,10 @@ GEMM_CASES = [
     (1, 64, 32, 2),
     (5000, 3072, 256, 4),        # the drift workload's shape, fewer tokens
     (300, 4096, 256, 8),
+    (1000, 192, 160, 5),         # one epilogue group (N_r % 64 != 0), 5 slots
+    (600, 320, 192, 6),          # two groups of 96 experts
+    (513, 64, 224, 7),           # one group of 224 experts, a single K stage
+    (2 * 128 * 148 + 5, 128, 64, 2),  # more pair tiles than the persistent grid holds at once
 ]
 
 
