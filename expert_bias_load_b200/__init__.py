@@ -23,8 +23,8 @@ import torch
 __all__ = [
     "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_logits", "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
-    "read_internal_status", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD", "EBL_ST_TIMEOUT",
-    "EBL_ST_BAD_COUNTS",
+    "read_internal_status", "check_finite", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD",
+    "EBL_ST_TIMEOUT", "EBL_ST_BAD_COUNTS", "EBL_ST_NONFINITE",
     "SMEBU_LAMBDA", "SMEBU_BETA", "SMEBU_KAPPA",
 ]
 
@@ -33,6 +33,7 @@ lib_path = os.path.join(_HERE, "libebl.so")
 
 EBL_OK, EBL_EINVAL, EBL_EUNSUPPORTED, EBL_ECUDA, EBL_EDATA = 0, -1, -2, -3, -4
 EBL_ST_BAD_EXPERT, EBL_ST_BAD_DEST, EBL_ST_EMPTY_LOAD, EBL_ST_TIMEOUT, EBL_ST_BAD_COUNTS = 1, 2, 4, 8, 16
+EBL_ST_NONFINITE = 32
 
 # Trinity Large's SMEBU constants ("Arcee Trinity Large Technical Report" 2.3)
 SMEBU_LAMBDA, SMEBU_BETA, SMEBU_KAPPA = 5e-4, 0.5, 2.0
@@ -59,7 +60,9 @@ SIGNATURES = {
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "ebl_read_internal_status": (_I, [_P, _I]),
     "ebl_selftest_wait_timeout": (_I, [_P, ctypes.c_uint, _P]),
-    "ebl_selftest_score_error": (_I, [_P, ctypes.c_int64, _P, _P, _P]),
+    "ebl_selftest_score_error": (_I, [_P, ctypes.c_int64, _P, _P, _P, _P]),
+    "ebl_check_finite_f32": (_I, [_P, ctypes.c_int64, _P, _P]),
+    "ebl_check_finite_bf16": (_I, [_P, ctypes.c_int64, _P, _P]),
 }
 
 
@@ -282,14 +285,29 @@ def selftest_wait_timeout(status, limit_us=20000, stream=None):
     _call("ebl_selftest_wait_timeout", _ptr(status), int(limit_us), _stream(stream))
 
 
-def selftest_score_error(x, max_err=None, stream=None):
+def selftest_score_error(x, max_err=None, exact_out=None, stream=None):
     """Largest distance between the approximate score logits mode ranks with
     and the exact one over the fp32 values in x (device), and the error bound
-    that ranking assumes.  Returns (max_err as a float, bound)."""
+    that ranking assumes.  Returns (max_err as a float, bound).  If exact_out
+    (fp32, same size as x) is given it receives the exact scores."""
     _check(x, "x", torch.float32)
     if max_err is None:
         max_err = torch.empty(1, dtype=torch.float32, device=x.device)
     _check(max_err, "max_err", torch.float32, (1,))
+    if exact_out is not None:
+        _check(exact_out, "exact_out", torch.float32, tuple(x.shape))
     bound = ctypes.c_float(0.0)
-    _call("ebl_selftest_score_error", _ptr(x), int(x.numel()), _ptr(max_err), ctypes.c_void_p(ctypes.addressof(bound)), _stream(stream))
+    _call("ebl_selftest_score_error", _ptr(x), int(x.numel()), _ptr(max_err),
+          ctypes.c_void_p(ctypes.addressof(bound)), _ptr(exact_out), _stream(stream))
     return float(max_err.item()), float(bound.value)
+
+
+def check_finite(x, status, stream=None):
+    """OR EBL_ST_NONFINITE into status (int32 [1]) if the fp32 or bf16 tensor x
+    holds a NaN or an infinity."""
+    _check(status, "status", torch.int32, (1,))
+    if not isinstance(x, torch.Tensor) or x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be a float32 or bfloat16 tensor")
+    _check(x, "x", x.dtype)
+    name = "ebl_check_finite_f32" if x.dtype == torch.float32 else "ebl_check_finite_bf16"
+    _call(name, _ptr(x), int(x.numel()), _ptr(status), _stream(stream))

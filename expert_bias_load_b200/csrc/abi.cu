@@ -284,6 +284,25 @@ int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *d
     return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
+static int check_finite_call(const void *x, int64_t n, int bf16, int32_t *status, ebl_stream_t stream) {
+    if (n < 0 || !status || !aligned4(status)) return EBL_EINVAL;
+    if (n > 0 && (!x || (reinterpret_cast<uintptr_t>(x) & (bf16 ? 1u : 3u)))) return EBL_EINVAL;
+    if (n == 0) return EBL_OK;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    cudaError_t e = ebl::launch_check_finite(x, n, bf16, status, di.num_sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
+}
+
+int ebl_check_finite_f32(const float *x, int64_t n, int32_t *status, ebl_stream_t stream) {
+    return check_finite_call(x, n, 0, status, stream);
+}
+
+int ebl_check_finite_bf16(const uint16_t *x, int64_t n, int32_t *status, ebl_stream_t stream) {
+    return check_finite_call(x, n, 1, status, stream);
+}
+
 int ebl_read_internal_status(int32_t *out, int clear) {
     if (!out) return EBL_EINVAL;
     DeviceInfo di;

@@ -568,10 +568,14 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
 
 // max over i of |approximate score - exact score| as the bits of a
 // non-negative float (those order like unsigned integers)
-__global__ void score_error_kernel(const float *__restrict__ x, int64_t n, unsigned *__restrict__ max_bits) {
+__global__ void score_error_kernel(const float *__restrict__ x, int64_t n, unsigned *__restrict__ max_bits,
+                                   float *__restrict__ exact_out) {
     float worst = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        worst = fmaxf(worst, fabsf(key_approx(x[i], 0.5f) - sigmoid_rounded_once(x[i])));
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float e = sigmoid_rounded_once(x[i]);
+        worst = fmaxf(worst, fabsf(key_approx(x[i], 0.5f) - e));
+        if (exact_out) exact_out[i] = e;
+    }
     atomicMax(max_bits, __float_as_uint(worst));
 }
 
@@ -679,13 +683,13 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
     return cudaGetLastError();
 }
 
-cudaError_t launch_score_error(const float *x, int64_t n, float *max_err, cudaStream_t stream) {
+cudaError_t launch_score_error(const float *x, int64_t n, float *max_err, float *exact_out, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(max_err, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     if (n == 0) return cudaSuccess;
     int64_t blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    score_error_kernel<<<(int)blocks, 256, 0, stream>>>(x, n, reinterpret_cast<unsigned *>(max_err));
+    score_error_kernel<<<(int)blocks, 256, 0, stream>>>(x, n, reinterpret_cast<unsigned *>(max_err), exact_out);
     return cudaGetLastError();
 }
 

@@ -39,12 +39,13 @@ extern "C" int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us,
     return EBL_OK;
 }
 
-extern "C" int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound,
+extern "C" int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound, float *exact_out,
                                         ebl_stream_t stream) {
     if (n < 0 || !max_err || (reinterpret_cast<uintptr_t>(max_err) & 3u)) return EBL_EINVAL;
     if (n > 0 && (!x || (reinterpret_cast<uintptr_t>(x) & 3u))) return EBL_EINVAL;
+    if (exact_out && (reinterpret_cast<uintptr_t>(exact_out) & 3u)) return EBL_EINVAL;
     if (bound) *bound = ebl::logits_key_error_bound();
-    if (ebl::launch_score_error(x, n, max_err, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (ebl::launch_score_error(x, n, max_err, exact_out, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return EBL_ECUDA;
     return EBL_OK;
 }

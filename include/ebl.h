@@ -59,6 +59,7 @@ typedef struct CUstream_st *ebl_stream_t;
 #define EBL_ST_EMPTY_LOAD 4   /* sum of loads was 0: bias/momentum left untouched */
 #define EBL_ST_TIMEOUT 8      /* a pipeline wait inside the router kernel ran out; outputs invalid */
 #define EBL_ST_BAD_COUNTS 16  /* dispatch: tile_counts do not add up to T*K (they do not match topk_idx) */
+#define EBL_ST_NONFINITE 32   /* ebl_check_finite_*: a NaN or infinity was found */
 
 #define EBL_MAX_EXPERTS 256   /* N_r limit of every entry point */
 #define EBL_MAX_TOPK 8        /* K limit */
@@ -297,10 +298,24 @@ int ebl_selftest_wait_timeout(int32_t *status, unsigned int limit_us, ebl_stream
  * largest; the bound must exceed the approximation's error.  This call writes
  *   *max_err = max_i | approx(x_i) - (float)(1 / (1 + exp(-(double)x_i))) |
  * (device fp32, 4-byte aligned) and, if bound is not NULL, the absolute error
- * bound the ranking assumes to *bound (host).  x: device fp32 [n], n >= 0.
+ * bound the ranking assumes to *bound (host).  If exact_out is not NULL
+ * (device fp32 [n]) it receives the exact scores (float)(1/(1+exp(-(double)x_i)))
+ * as this library computes them, so that they can be compared with another
+ * fp64 implementation.  x: device fp32 [n], n >= 0.
  * No counterpart on the pages: it tests an implementation assumption.
  */
-int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound, ebl_stream_t stream);
+int ebl_selftest_score_error(const float *x, int64_t n, float *max_err, float *bound, float *exact_out,
+                             ebl_stream_t stream);
+
+/*
+ * ebl_check_finite_f32 / ebl_check_finite_bf16 -- input validation.  The
+ * router assumes finite logits, hidden states and bias; these scan n values
+ * (device, 4-byte aligned for fp32, 2-byte for bf16) and OR EBL_ST_NONFINITE
+ * into *status (device int32, not NULL) if any is NaN or +-inf.  One read of
+ * the buffer; asynchronous on the stream.  No counterpart on the pages.
+ */
+int ebl_check_finite_f32(const float *x, int64_t n, int32_t *status, ebl_stream_t stream);
+int ebl_check_finite_bf16(const uint16_t *x, int64_t n, int32_t *status, ebl_stream_t stream);
 
 /*
  * ebl_read_internal_status -- copy the library-owned status word (used when a

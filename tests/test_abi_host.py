@@ -90,9 +90,15 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.moe_combine(FAKE, FAKE, FAKE, 100, 64, 9, FAKE, None, None) == EINVAL
     assert lib.moe_combine(FAKE, FAKE, FAKE, 0, 64, 2, FAKE, None, None) == 0
     assert lib.ebl_read_internal_status(None, 0) == EINVAL
-    assert lib.ebl_selftest_score_error(FAKE, -1, FAKE, None, None) == EINVAL
-    assert lib.ebl_selftest_score_error(FAKE, 10, None, None, None) == EINVAL
-    assert lib.ebl_selftest_score_error(None, 10, FAKE, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(FAKE, -1, FAKE, None, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(FAKE, 10, None, None, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(None, 10, FAKE, None, None, None) == EINVAL
+    assert lib.ebl_selftest_score_error(FAKE, 10, FAKE, None, ctypes.c_void_p(0x10002), None) == EINVAL
+    assert lib.ebl_check_finite_f32(FAKE, -1, FAKE, None) == EINVAL
+    assert lib.ebl_check_finite_f32(FAKE, 10, None, None) == EINVAL
+    assert lib.ebl_check_finite_f32(ctypes.c_void_p(0x10002), 10, FAKE, None) == EINVAL   # not 4-byte aligned
+    assert lib.ebl_check_finite_bf16(ctypes.c_void_p(0x10001), 10, FAKE, None) == EINVAL  # not 2-byte aligned
+    assert lib.ebl_check_finite_bf16(None, 0, FAKE, None) == 0                              # empty: nothing to do
 
 
 def test_binding_has_no_cpu_fallback():
