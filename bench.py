@@ -247,6 +247,20 @@ def oracle_suite_cpu(seconds):
         t = run(rows, 2)
         out.append({"workload": name, "mode": mode, "rows": rows, "seconds": t, "tokens_per_s": rows / t,
                     "extrapolated": rows < T})
+    # the bias updates alone, per step, at N_r = 256 on the tie workload's loads
+    counts = np.bincount(np.random.default_rng(5).integers(0, 256, 4 * 1048576), minlength=256).astype(np.int64)
+    b = synth.dead_start_bias(256).numpy()
+    m = np.zeros(256, np.float32)
+    reps = 2000
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.smebu(counts, b, m)
+    t_smebu = (time.perf_counter() - t0) / reps
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.sign_update(counts, b)
+    t_sign = (time.perf_counter() - t0) / reps
+    out.append({"workload": "ties", "mode": "updates", "smebu_us": t_smebu * 1e6, "sign_us": t_sign * 1e6})
     return out
 
 
@@ -277,6 +291,19 @@ def oracle_suite(args):
         return ev[0].elapsed_time(ev[1]) / reps
 
     entries = []
+    # bias updates alone: one CTA per step; 1000 back-to-back launches per CUDA-event pair
+    counts = torch.bincount(torch.randint(0, 256, (4 * 1048576,), generator=torch.Generator().manual_seed(5)),
+                            minlength=256).to(torch.int32).to(dev)
+    b = synth.dead_start_bias(256, device=dev)
+    m = torch.zeros(256, device=dev)
+    upd = {"workload": "ties", "step": "bias update alone (N_r = 256)",
+           "gpu_smebu_us": gpu_ms(lambda: ebl.smebu_step(counts, b, m), reps=1000) * 1e3,
+           "gpu_sign_us": gpu_ms(lambda: ebl.sign_update_step(counts, b, 1e-3), reps=1000) * 1e3,
+           "note": "GPU per launch from Python: the host's launch rate bounds it (the kernel itself takes about "
+                   "5 us in a launch list)"}
+    for label, (threads, res) in cpu.items():
+        upd["oracle_" + label + "_smebu_us"] = res[-1]["smebu_us"]
+        upd["oracle_" + label + "_sign_us"] = res[-1]["sign_us"]
     for i, (name, mode) in enumerate(SUITE_ENTRIES):
         c = synth.WORKLOADS[name]
         T, d, Nr, K = c["T"], c["d"], c["Nr"], c["K"]
@@ -328,6 +355,7 @@ def oracle_suite(args):
         entries.append(e)
         del fn
         torch.cuda.empty_cache()
+    entries.append(upd)
     print(json.dumps({"oracle_suite": entries, "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
                       "note": "oracle samples sized for about %.0f s each; a sample smaller than T is "
                               "extrapolated linearly" % args.cpu_seconds}), flush=True)

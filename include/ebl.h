@@ -57,7 +57,7 @@ typedef struct CUstream_st *ebl_stream_t;
 #define EBL_ST_BAD_EXPERT 1   /* an expert id outside [0, N_r) was seen; that pair was skipped */
 #define EBL_ST_BAD_DEST 2     /* a dest index outside [0, T*K) was seen; that slot was skipped */
 #define EBL_ST_EMPTY_LOAD 4   /* sum of loads was 0: bias/momentum left untouched */
-#define EBL_ST_TIMEOUT 8      /* a pipeline wait inside the router kernel ran out; outputs invalid */
+#define EBL_ST_TIMEOUT 8      /* a pipeline wait (router kernel, dispatch copy) ran out; outputs invalid */
 #define EBL_ST_BAD_COUNTS 16  /* dispatch: tile_counts do not add up to T*K (they do not match topk_idx) */
 #define EBL_ST_NONFINITE 32   /* ebl_check_finite_*: a NaN or infinity was found */
 
@@ -221,8 +221,11 @@ int sign_update_step(int32_t *counts, float *bias, int N_r, float gamma, int res
  *              skipped and its dest is -1.  EBL_ST_BAD_COUNTS if the given
  *              tile_counts do not add up to T*K; destinations that would fall
  *              outside [0, T*K) are then skipped (dest -1), others are not
- *              meaningful.  Nothing is written outside the output buffers.
- * T*K <= 2^31 - 1.
+ *              meaningful.  EBL_ST_TIMEOUT if a row copy did not complete
+ *              within the bounded wait (dispatched rows are then not valid).
+ *              Nothing is written outside the output buffers.
+ * The rows move by TMA bulk copies through shared memory (one read of each
+ * hidden row, one write per destination).  T*K <= 2^31 - 1.
  */
 size_t ebl_dispatch_workspace_bytes(int T, int N_r);
 int moe_dispatch(const uint16_t *hidden, const int32_t *topk_idx, const int32_t *tile_counts,
