@@ -46,6 +46,9 @@ LOGITS_CASES = [
     (500, 68, 6, False, "small"),        # just past 64 experts: 4 float4 per lane, 3 of them partly padding
     (500, 132, 3, True, "dead"),         # just past 128: 8 float4 per lane
     (600, 252, 8, True, "ties"),         # ragged last column block
+    (100, 1, 1, False, "small"),         # a single expert
+    (257, 2, 2, True, "ties"),           # K = N_r with ties
+    (300, 3, 2, True, "ties"),
 ]
 
 
