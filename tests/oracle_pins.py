@@ -18,6 +18,10 @@ What pins what:
     constant counts, step bounds.
   - Sign update: closed-form trajectory, zero-mean bias, sign(0) = 0.
   - MaxVio: hand examples (golden/maxvio.txt).
+  - Per-tile loads (logits mode): numpy bincount of each 128-token tile's
+    selections, summing to the per-expert counts.
+  - The near-tie gap that GEMM-mode parity uses to excuse tokens: the K-th
+    minus the (K+1)-th largest biased score, from a numpy sort of the scores.
   - Dispatch: numpy stable argsort; permutation and offset invariants.
   - Combine: numpy einsum in fp64; the identity-expert round trip; the fp32
     chain within its rounding bound.
@@ -148,6 +152,35 @@ def pin_zero_bias_is_topk_of_logits():
     rl = oracle.router_logits(xl, np.zeros(Nr, np.float32), K)
     refl = torch.topk(torch.from_numpy(xl.astype(np.float64)), K, dim=1, sorted=True).indices.numpy()
     assert np.array_equal(rl.idx, refl.astype(np.int32))
+
+
+def pin_tile_counts_are_tile_histograms():
+    rng = np.random.default_rng(29)
+    T, Nr, K, tile = 1000, 16, 3, 128           # a ragged last tile
+    x = rng.standard_normal((T, Nr)).astype(np.float32)
+    b = (rng.standard_normal(Nr) * 0.1).astype(np.float32)
+    r = oracle.router_logits(x, b, K, tile_tokens=tile)
+    tiles = (T + tile - 1) // tile
+    assert r.tile_counts.shape == (tiles, Nr)
+    for j in range(tiles):
+        want = np.bincount(r.idx[j * tile:(j + 1) * tile].ravel(), minlength=Nr)
+        assert np.array_equal(r.tile_counts[j], want), j
+    assert np.array_equal(r.tile_counts.sum(0), r.counts)
+
+
+def pin_gap_is_kth_minus_next_biased_score():
+    rng = np.random.default_rng(31)
+    T, d, Nr, K = 200, 64, 24, 5
+    h = _bf16(rng.standard_normal((T, d)))
+    w = _bf16(rng.standard_normal((Nr, d)) * 0.2)
+    b = (rng.standard_normal(Nr) * 0.05).astype(np.float32)
+    r = oracle.router_gemm(h, w, b, K, want_scores=True)
+    keys = np.sort(r.scores + b.astype(np.float64), axis=1)[:, ::-1]
+    want = keys[:, K - 1] - keys[:, K]
+    assert np.all(r.gap >= 0)
+    assert np.allclose(r.gap, want, rtol=0, atol=1e-15)
+    rk = oracle.router_gemm(h, w, b, Nr)        # K = N_r: nothing is left out
+    assert np.all(np.isinf(rk.gap))
 
 
 def pin_bias_forces_expert():

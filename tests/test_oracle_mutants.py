@@ -4,7 +4,8 @@ Each case below alters one line of a copy of oracle/ebl_oracle.c the way a
 plausible slip would (a flipped sign, a dropped term, a swapped coefficient, a
 transposed operand, a reversed tie-break, ...), compiles the copy, and runs the
 pins against it: at least one pin has to fail.  The oracle itself is never
-modified.
+modified.  Every planted mistake keeps the copy's memory accesses in bounds,
+because the copies run inside the test process.
 """
 import os
 
@@ -54,6 +55,12 @@ MUTANTS = {
     "dispatch_unstable": ("    for (int64_t p = 0; p < P; ++p) {\n        int e = idx[p];",
                           "    for (int64_t p = P - 1; p >= 0; --p) {\n        int e = idx[p];"),
     "dispatch_perm_pair": ("perm[j] = (int32_t)(p / K);", "perm[j] = (int32_t)(p % T);"),
+    "tile_counts_first_slot": ("tile_counts[(p / K / tile_tokens) * Nr + idx[p]] += 1;",
+                               "tile_counts[(p / K / tile_tokens) * Nr + idx[p - p % K]] += 1;"),
+    "gap_sign": ("gap_out[t] = (K == Nr) ? INFINITY : key[sel[K - 1]] - best_rest;",
+                 "gap_out[t] = (K == Nr) ? INFINITY : best_rest - key[sel[K - 1]];"),
+    "gap_from_first_slot": ("gap_out[t] = (K == Nr) ? INFINITY : key[sel[K - 1]] - best_rest;",
+                            "gap_out[t] = (K == Nr) ? INFINITY : key[sel[0]] - best_rest;"),
     "combine_drops_slot": ("            for (int k = 0; k < K; ++k) {\n                const int64_t row",
                            "            for (int k = 0; k < K - 1; ++k) {\n                const int64_t row"),
 }
