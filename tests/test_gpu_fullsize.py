@@ -12,7 +12,7 @@ from tests.parity import assert_gemm_parity, to_np
 
 pytestmark = pytest.mark.gpu
 
-SAMPLE_ROWS = 2048
+SAMPLE_ROWS = 8192
 
 
 def _sampled_parity(h_dev, W, bias, K, idx, gates, seed):
@@ -21,9 +21,9 @@ def _sampled_parity(h_dev, W, bias, K, idx, gates, seed):
     rows = torch.randperm(T, generator=g)[:SAMPLE_ROWS]
     rows = torch.cat([rows, torch.tensor([0, T - 1])]).sort().values
     hs = h_dev[rows.to(h_dev.device)].cpu()
-    ref = oracle.router_gemm(hs, W.cpu(), bias.cpu().numpy(), K)
+    ref = oracle.router_gemm(hs, W.cpu(), bias.cpu().numpy(), K, want_scores=True)
     r = rows.numpy()
-    return assert_gemm_parity(to_np(idx)[r], to_np(gates)[r], ref, W.shape[0])
+    return assert_gemm_parity(to_np(idx)[r], to_np(gates)[r], ref, W.shape[0], bias.cpu().numpy())
 
 
 @pytest.mark.parametrize("name", ["mid", "drift", "ties"])

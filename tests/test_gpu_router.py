@@ -126,9 +126,9 @@ def test_gemm_mode_vs_oracle(cuda_device, T, d, Nr, K):
                                     status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    ref = oracle.router_gemm(h, W, bias.numpy(), K)
+    ref = oracle.router_gemm(h, W, bias.numpy(), K, want_scores=True)
     gi = to_np(idx)
-    assert_gemm_parity(gi, to_np(gates), ref, Nr, gpu_counts=to_np(counts))
+    assert_gemm_parity(gi, to_np(gates), ref, Nr, bias.numpy(), gpu_counts=to_np(counts))
     assert np.array_equal(to_np(tiles), tile_hist(gi, Nr))
     g = to_np(gates).astype(np.float64)
     assert np.allclose(g.sum(1), 1.0, atol=K * 2e-7)
@@ -148,11 +148,11 @@ def test_gemm_mode_tiny_workload_smebu_steps(cuda_device):
     maxvio = torch.zeros(1, device=dev)
     for step in range(cfg["steps"]):
         h = synth.hidden_normal(T, d, seed=synth.step_seed("tiny", step))
-        ref = oracle.router_gemm(h, W, b_o, K)
+        ref = oracle.router_gemm(h, W, b_o, K, want_scores=True)
         idx, gates = ebl.router_forward(h.to(dev), W.to(dev), b_g, K, counts)
         torch.cuda.synchronize()
         n_gpu = to_np(counts).astype(np.int64)
-        assert_gemm_parity(to_np(idx), to_np(gates), ref, Nr, gpu_counts=n_gpu)
+        assert_gemm_parity(to_np(idx), to_np(gates), ref, Nr, b_o, gpu_counts=n_gpu)
         ebl.smebu_step(counts, b_g, m_g, reset_counts=True, maxvio=maxvio)
         # open loop: the oracle's SMEBU is fed the GPU's counts
         oracle.smebu(n_gpu, b_o, m_o)
