@@ -181,3 +181,40 @@ def test_full_step_in_cuda_graph(cuda_device):
         state[mode] = (b.clone(), m.clone(), idx.clone(), dest.clone(), X.clone(), out.clone())
     for a, c in zip(state["eager"], state["graph"]):
         assert torch.equal(a, c)
+
+
+def test_closed_loop_gemm_drift_is_reported(cuda_device):
+    """GEMM mode, closed loop on both sides: the library and the oracle each
+    route with their own bias and update it from their own counts for 20 SMEBU
+    steps (8192 tokens of the mid workload's shape per step).  Near-tie tokens
+    may differ by a count or two, so the trajectories are reported, not
+    compared against a tolerance; what the equations fix is asserted on both
+    sides (sum of b stays 0, |m| <= 2 lambda)."""
+    import numpy as np
+    import oracle
+    dev = cuda_device
+    cfg = synth.WORKLOADS["mid"]
+    T, d, Nr, K, steps = 8192, cfg["d"], cfg["Nr"], cfg["K"], 20
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d)
+    b_g = torch.zeros(Nr, device=dev)
+    m_g = torch.zeros(Nr, device=dev)
+    b_o = np.zeros(Nr, np.float32)
+    m_o = np.zeros(Nr, np.float32)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    drift, count_diff = [], []
+    for s in range(steps):
+        h = synth.hidden_normal(T, d, seed=synth.step_seed("mid", s))
+        ebl.router_forward(h.to(dev), W.to(dev), b_g, K, counts)
+        n_g = counts.cpu().numpy().astype(np.int64)
+        ebl.smebu_step(counts, b_g, m_g, reset_counts=True)
+        r = oracle.router_gemm(h, W, b_o, K)
+        oracle.smebu(r.counts, b_o, m_o)
+        bg = b_g.cpu().numpy()
+        drift.append(float(np.abs(bg.astype(np.float64) - b_o).max()))
+        count_diff.append(int(np.abs(n_g - r.counts).sum()))
+        for b, m in ((bg, m_g.cpu().numpy()), (b_o, m_o)):
+            assert abs(float(b.astype(np.float64).sum())) <= 1e-4
+            assert float(np.abs(m).max()) <= 2 * 5e-4 * (1 + 1e-6)
+    print("\nclosed-loop GEMM mode, mid shape, 8192 tokens/step: max |b_gpu - b_oracle| per step")
+    print(json.dumps([float("%.3g" % x) for x in drift]))
+    print("sum |n_gpu - n_oracle| per step:", count_diff)
