@@ -273,7 +273,7 @@ constexpr size_t vec_ring_bytes() {
     return sizeof(float) * kWarpsPerCta * kStages * kRowsPerGroup * 32 * NV;
 }
 
-template <int K, int NV>
+template <int K, int NV, bool FULL>
 __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float *__restrict__ logits,
                                                                      const float *__restrict__ bias, int T, int Nr,
                                                                      int32_t *__restrict__ topk_idx,
@@ -283,6 +283,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     // lane-local lists of the approximate pass hold P >= K values (P a power of two)
     constexpr int P = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
     constexpr int kRow = 32 * NV;  // floats per row in the ring (N_r rounded up, zero-filled)
+    // FULL: N_r == kRow, so every column a lane copies exists (no per-column test)
     static_assert(NV % 2 == 0 && kRow <= kMaxExperts, "a lane holds NV float4 of a row, in pairs");
     extern __shared__ __align__(16) float ring_s[];  // [warp][stage][row of group][kRow]
     __shared__ __align__(16) float hb_s[kMaxExperts];  // fl(0.5 + b); -inf past N_r
@@ -336,30 +337,34 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         const int64_t tile = (int64_t)blockIdx.x + (int64_t)(item >> 3) * gridDim.x;
         return tile * kTileTokens + warp * 32 + (item & 7) * kRowsPerGroup + r;
     };
-    auto issue = [&](int item) {
-        const int64_t row = item_row(item);
+    auto issue = [&](int item, int64_t row) {
         const bool rin = row < T;
         const float *src = logits + (rin ? row : 0) * (int64_t)Nr;
         float *dst = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;
 #pragma unroll
         for (int m = 0; m < NV; ++m) {
             const int c = 4 * (8 * m + j);
-            const bool ok = rin && c < Nr;
+            const bool ok = FULL ? rin : (rin && c < Nr);
             cp_async_16(dst + c, src + (ok ? c : 0), ok);
         }
         cp_async_commit();
     };
+    // the row of item + 1 from the row of item (the same tile, or the next tile of this CTA)
+    const int64_t tile_jump = (int64_t)gridDim.x * kTileTokens - (kGroupsPerWarp - 1) * kRowsPerGroup;
+    auto next_row = [&](int64_t row, int item) { return ((item + 1) & 7) ? row + kRowsPerGroup : row + tile_jump; };
 
     const int items = num_tiles > (int)blockIdx.x
                           ? ((num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * kGroupsPerWarp
                           : 0;
-#pragma unroll
-    for (int q = 0; q < kStages - 1; ++q) issue(q);
+    static_assert(kStages == 2, "one item in flight while one is ranked");
+    int64_t ahead = item_row(0);  // the row of the most recently issued item
+    issue(0, ahead);
     for (int item = 0; item < items; ++item) {
-        issue(item + kStages - 1);  // into the stage the previous item released
+        const int64_t row = ahead;
+        ahead = next_row(ahead, item);
+        issue(item + 1, ahead);  // into the stage the previous item released
         cp_async_wait<kStages - 1>();
         __syncwarp();
-        const int64_t row = item_row(item);
         const float *xr = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;  // this lane's row
 
         // approximate keys of this lane's 4*NV experts
@@ -618,10 +623,10 @@ cudaError_t vec_setup(const void *kern, size_t smem, int *blocks_per_sm) {
     return cudaSuccess;
 }
 
-template <int K, int NV>
+template <int K, int NV, bool FULL>
 cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, int32_t *topk_idx, float *gates,
                        int32_t *counts, int32_t *tile_counts, int num_sms, cudaStream_t stream) {
-    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV>);
+    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL>);
     const size_t smem = vec_ring_bytes<NV>();
     int per_sm = 1;
     cudaError_t err = vec_setup(kern, smem, &per_sm);
@@ -629,8 +634,8 @@ cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, in
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     int grid = num_sms * per_sm;
     if (grid > num_tiles) grid = num_tiles;
-    router_logits_vec_kernel<K, NV><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates, counts,
-                                                                      tile_counts);
+    router_logits_vec_kernel<K, NV, FULL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates,
+                                                                            counts, tile_counts);
     return cudaGetLastError();
 }
 
@@ -646,7 +651,9 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
         switch (K * 16 + nv) {
 #define EBL_VCASE(KK, NN) \
     case KK * 16 + NN:    \
-        return launch_vec<KK, NN>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream);
+        return Nr == 32 * NN                                                                                   \
+                   ? launch_vec<KK, NN, true>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream) \
+                   : launch_vec<KK, NN, false>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream);
 #define EBL_VCASES(KK) EBL_VCASE(KK, 2) EBL_VCASE(KK, 4) EBL_VCASE(KK, 8)
             EBL_VCASES(1)
             EBL_VCASES(2)
