@@ -125,8 +125,10 @@ int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float
  * table); "Arcee Trinity Large Technical Report" section 6 gives its weight
  * (1e-4 intended, 1e-6 effective).  The mean z-loss is zloss_sum / T.  The
  * log-sum-exp is formed from the fp32 logits around the row maximum (no
- * overflow).  zloss_sum: device, 8-byte aligned, not NULL.  Other arguments
- * and outputs as router_forward.
+ * overflow).  zloss_sum: device, 8-byte aligned, not NULL.  The per-warp
+ * partial sums meet in fp64 atomics, so the last bits of zloss_sum can vary
+ * between runs with the order in which CTAs finish; indices, gates and counts
+ * stay deterministic.  Other arguments and outputs as router_forward.
  */
 int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const float *bias,
                          int T, int d, int N_r, int K,
