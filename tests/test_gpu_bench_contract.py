@@ -41,3 +41,10 @@ def test_bench_line_has_the_contract_keys(cuda_device):
     assert e["h2d_bytes_per_step"] == 65536 * 4096 * 2 and e["d2h_bytes_per_step"] > 0 and e["value"] > 0
     assert j["gpu_launches"] == 2 * 5
     assert "sm_mhz" in j["clocks"] and "reasons" in j["clocks"]
+
+
+def test_smoke_entry_point(cuda_device):
+    """__graft_entry__.smoke() runs as the round-end check runs it."""
+    sys.path.insert(0, ROOT)
+    import __graft_entry__
+    __graft_entry__.smoke()
