@@ -134,3 +134,23 @@ def test_dispatch_inconsistent_tile_counts_sets_status(cuda_device):
     dn = to_np(dest)
     assert np.all((dn == -1) | ((dn >= 0) & (dn < T * K)))
     assert torch.all(guard == 7)
+
+
+@pytest.mark.parametrize("T,d,K", [(1000, 1024, 4), (333, 136, 3), (64, 8, 8), (257, 4096, 1)])
+def test_combine_distinct_expert_outputs_vs_oracle(cuda_device, T, d, K):
+    """Every slot of a token reads a different expert-output row (random rows,
+    a random permutation as dest, gates that do not sum to 1), so a slot read
+    from the wrong row or a dropped slot changes the result; bit-exact against
+    the oracle's fp32 fma chain in slot order."""
+    dev = cuda_device
+    g0 = torch.Generator().manual_seed(T + d + K)
+    Y = synth.hidden_normal(T * K, d, seed=T * 3 + K)
+    dest = torch.randperm(T * K, generator=g0).to(torch.int32)
+    gates = (torch.rand(T, K, generator=g0) * 2.0 - 0.5).float()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = ebl.moe_combine(Y.to(dev), gates.to(dev), dest.to(dev), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    yb = Y.view(torch.int16).numpy().view(np.uint16)
+    _, o32 = oracle.combine(yb, gates.numpy(), dest.numpy())
+    assert np.array_equal(to_np(out).view(np.uint32), o32.view(np.uint32))
