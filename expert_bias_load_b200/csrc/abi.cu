@@ -121,7 +121,8 @@ int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const flo
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
     if (d < 64 || d > (1 << 20) || d % 64 != 0) return EBL_EINVAL;
     if (N_r % 32 != 0) return EBL_EUNSUPPORTED;
-    if (!hidden || !W_router || !bias || !topk_idx || !gates || !counts) return EBL_EINVAL;
+    if (!W_router || !bias || !counts) return EBL_EINVAL;
+    if (T > 0 && (!hidden || !topk_idx || !gates)) return EBL_EINVAL;  // T-sized buffers may be NULL when T == 0
     if (!aligned16(hidden) || !aligned16(W_router) || !aligned4(bias) || !aligned4(counts)) return EBL_EINVAL;
     if (K % 4 == 0 && (!aligned16(topk_idx) || !aligned16(gates))) return EBL_EINVAL;
     if (!aligned4(topk_idx) || !aligned4(gates) || (tile_counts && !aligned4(tile_counts))) return EBL_EINVAL;
@@ -188,7 +189,8 @@ int router_forward_logits(const float *logits, const float *bias, int T, int N_r
                           ebl_stream_t stream) {
     (void)status;  // no device-side error condition in this mode
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
-    if (!logits || !bias || !topk_idx || !gates || !counts) return EBL_EINVAL;
+    if (!bias || !counts) return EBL_EINVAL;
+    if (T > 0 && (!logits || !topk_idx || !gates)) return EBL_EINVAL;  // T-sized buffers may be NULL when T == 0
     if (!aligned4(logits) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(gates) || !aligned4(counts))
         return EBL_EINVAL;
     if (tile_counts && !aligned4(tile_counts)) return EBL_EINVAL;
@@ -248,7 +250,8 @@ int moe_dispatch(const uint16_t *hidden, const int32_t *topk_idx, const int32_t 
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
     if ((long long)T * K > 2147483647LL) return EBL_EINVAL;
     if (d < 8 || d % 8 != 0 || d > (1 << 24)) return EBL_EINVAL;
-    if (!hidden || !topk_idx || !offsets || !perm || !dest || !dispatched || !workspace) return EBL_EINVAL;
+    if (!offsets) return EBL_EINVAL;
+    if (T > 0 && (!hidden || !topk_idx || !perm || !dest || !dispatched || !workspace)) return EBL_EINVAL;
     if (!aligned16(hidden) || !aligned16(dispatched) || !aligned16(workspace)) return EBL_EINVAL;
     if (!aligned4(topk_idx) || !aligned4(offsets) || !aligned4(perm) || !aligned4(dest)) return EBL_EINVAL;
     if (tile_counts && !aligned4(tile_counts)) return EBL_EINVAL;
@@ -272,7 +275,7 @@ int moe_combine(const uint16_t *expert_out, const float *gates, const int32_t *d
     if (check_T(T) || K < 1 || K > EBL_MAX_TOPK) return EBL_EINVAL;
     if ((long long)T * K > 2147483647LL) return EBL_EINVAL;
     if (d < 8 || d % 8 != 0 || d > (1 << 24)) return EBL_EINVAL;
-    if (!expert_out || !gates || !dest || !out) return EBL_EINVAL;
+    if (T > 0 && (!expert_out || !gates || !dest || !out)) return EBL_EINVAL;
     if (!aligned16(expert_out) || !aligned16(out) || !aligned4(gates) || !aligned4(dest)) return EBL_EINVAL;
     if (T == 0) return EBL_OK;
     DeviceInfo di;

@@ -71,7 +71,8 @@ extern "C" int moe_dispatch_static(const uint16_t *hidden, const int32_t *topk_i
     if (N_r < 1 || N_r > EBL_MAX_EXPERTS || K < 1 || K > EBL_MAX_TOPK || K > N_r) return EBL_EINVAL;
     if ((long long)T * K > 2147483647LL) return EBL_EINVAL;
     if (d < 8 || d % 8 != 0 || d > (1 << 24)) return EBL_EINVAL;
-    if (!hidden || !topk_idx || !offsets || !perm || !dest || !dispatched) return EBL_EINVAL;
+    if (!offsets) return EBL_EINVAL;
+    if (T > 0 && (!hidden || !topk_idx || !perm || !dest || !dispatched)) return EBL_EINVAL;
     if (!aligned16(hidden) || !aligned16(dispatched)) return EBL_EINVAL;
     if (!aligned4(topk_idx) || !aligned4(offsets) || !aligned4(perm) || !aligned4(dest)) return EBL_EINVAL;
     if (tile_counts && !aligned4(tile_counts)) return EBL_EINVAL;

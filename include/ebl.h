@@ -27,6 +27,8 @@
  *     is launched; a call that returns an error launched nothing, except
  *     EBL_ECUDA, which reports a launch failure.
  *   - Return value: EBL_OK (0) or a negative error code (ebl_strerror()).
+ *   - T == 0 (no tokens) is a no-op that launches nothing (moe_dispatch zeroes
+ *     offsets); the buffers whose size is proportional to T may then be NULL.
  *   - Errors only visible on the device (an expert id out of range, a sum of
  *     loads of zero, a pipeline wait that ran out) are OR-ed into the optional
  *     device word `status` as EBL_ST_* bits; kernels never trap.  With

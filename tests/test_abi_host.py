@@ -69,6 +69,14 @@ def test_router_forward_rejects_bad_arguments(lib):
     assert _router(lib, ptrs={"c": None}) == EINVAL
     assert _router(lib, ptrs={"h": ctypes.c_void_p(0x10008)}) == EINVAL   # not 16-byte aligned
     assert _router(lib, T=0) == 0                    # empty batch: nothing to do
+    # with no tokens the token-sized buffers may be NULL (empty tensors have no storage)
+    assert _router(lib, T=0, ptrs={"h": None, "i": None, "g": None}) == 0
+    assert _router(lib, T=0, ptrs={"w": None}) == EINVAL
+    assert _router(lib, T=1, ptrs={"i": None}) == EINVAL
+    assert lib.router_forward_logits(None, FAKE, 0, 8, 2, None, None, FAKE, None, None, None) == 0
+    assert lib.router_forward_logits(None, FAKE, 1, 8, 2, FAKE, FAKE, FAKE, None, None, None) == EINVAL
+    assert lib.moe_combine(None, None, None, 0, 64, 2, None, None, None) == 0
+    assert lib.moe_combine(None, FAKE, FAKE, 1, 64, 2, FAKE, None, None) == EINVAL
 
 
 def test_other_entry_points_reject_bad_arguments(lib):

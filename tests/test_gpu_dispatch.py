@@ -154,3 +154,27 @@ def test_combine_distinct_expert_outputs_vs_oracle(cuda_device, T, d, K):
     yb = Y.view(torch.int16).numpy().view(np.uint16)
     _, o32 = oracle.combine(yb, gates.numpy(), dest.numpy())
     assert np.array_equal(to_np(out).view(np.uint32), o32.view(np.uint32))
+
+
+def test_empty_batch_is_a_no_op(cuda_device):
+    """T = 0 through the binding (empty tensors have no storage): the router
+    modes and combine launch nothing and leave counts alone; dispatch zeroes
+    the offsets."""
+    dev = cuda_device
+    Nr, K, d = 64, 4, 256
+    counts = torch.arange(Nr, dtype=torch.int32, device=dev)
+    before = counts.clone()
+    W = synth.router_weight(Nr, d, seed=1).to(dev)
+    bias = torch.zeros(Nr, device=dev)
+    h = torch.empty(0, d, dtype=torch.bfloat16, device=dev)
+    idx, g = ebl.router_forward(h, W, bias, K, counts)
+    assert idx.shape == (0, K) and g.shape == (0, K)
+    idx, g = ebl.router_forward_logits(torch.empty(0, Nr, device=dev), bias, K, counts)
+    assert idx.shape == (0, K)
+    offsets, perm, dest, X = ebl.moe_dispatch(h, idx, Nr, offsets=torch.full((Nr + 1,), 7, dtype=torch.int32,
+                                                                             device=dev))
+    out = ebl.moe_combine(X, g, dest)
+    torch.cuda.synchronize()
+    assert torch.equal(counts, before)
+    assert int(offsets.abs().sum().item()) == 0
+    assert perm.numel() == 0 and X.shape == (0, d) and out.shape == (0, d)
