@@ -105,6 +105,9 @@ def _ptr(t):
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device.index != torch.cuda.current_device():
+        raise ValueError("stream is on %s but the current CUDA device is cuda:%d"
+                         % (stream.device, torch.cuda.current_device()))
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -115,6 +118,11 @@ def _check(t, name, dtype, shape=None):
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
     if not t.is_cuda:
         raise ValueError("%s must be on a CUDA device" % name)
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device; a tensor elsewhere would
+        # hand another GPU's pointer to its kernels
+        raise ValueError("%s is on %s but the current CUDA device is cuda:%d (use torch.cuda.device(...))"
+                         % (name, t.device, torch.cuda.current_device()))
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     if shape is not None and tuple(t.shape) != tuple(shape):
