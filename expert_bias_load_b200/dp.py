@@ -30,16 +30,24 @@ class DataParallelRouterStep:
 
     route(hidden, bias, counts) -> anything      accumulates local loads into counts
     update(counts, bias, momentum, maxvio)       bias update from global loads; resets counts
+
+    stream: the CUDA stream route and update run on, if not torch's current
+    one; the all-reduce is then issued on it too, so the three stay ordered.
     """
 
-    def __init__(self, route, update, group=None):
+    def __init__(self, route, update, group=None, stream=None):
         self.route = route
         self.update = update
         self.group = group
+        self.stream = stream
 
     def __call__(self, hidden, bias, momentum, counts, maxvio=None):
         out = self.route(hidden, bias, counts)
-        global_loads(counts, self.group)
+        if self.stream is not None:
+            with torch.cuda.stream(self.stream):
+                global_loads(counts, self.group)
+        else:
+            global_loads(counts, self.group)
         self.update(counts, bias, momentum, maxvio)
         return out
 
@@ -55,4 +63,4 @@ def cuda_step(W_router, K, lam=5e-4, beta=0.5, kappa=2.0, group=None, stream=Non
     def update(counts, bias, momentum, maxvio):
         ebl.smebu_step(counts, bias, momentum, lam, beta, kappa, reset_counts=True, maxvio=maxvio, stream=stream)
 
-    return DataParallelRouterStep(route, update, group)
+    return DataParallelRouterStep(route, update, group, stream)
