@@ -12,7 +12,7 @@
 // with a bounded distance to the exact one ranks all experts; the K-th largest
 // approximate key tau bounds the exact K-th key, and only experts whose
 // approximate key is within twice that distance of tau can be in the exact
-// Top-K.  Those candidates (usually K or K+1 per token) are scored exactly and
+// Top-K.  Those candidates (K to K+2 per token on most rows) are scored exactly and
 // the exact Top-K is taken among them: the same result as scoring every expert
 // in fp64.
 //
