@@ -1,7 +1,8 @@
 """Seeded random shapes through every mode against the oracle (small sizes):
 logits mode bit-exact (both kernels: aligned and misaligned logits), GEMM mode
-under the near-tie rule, dispatch and combine bit-exact.  Each case draws T,
-N_r, K, d, the bias pattern and the value distribution from its own seed."""
+under the near-tie rule, dispatch and combine bit-exact, and the bias updates
+(SMEBU clamped and linear over several layers, the sign update).  Each case
+draws its sizes, the bias pattern and the value distribution from its own seed."""
 import numpy as np
 import pytest
 import torch
@@ -109,3 +110,54 @@ def test_dispatch_combine_random_shapes(cuda_device, case):
     assert np.array_equal(to_np(X.view(torch.int16)).view(np.uint16), oracle.gather_rows(hb, o_perm))
     _, o32 = oracle.combine(Y.view(torch.int16).numpy().view(np.uint16), g, o_dest)
     assert np.array_equal(to_np(out).view(np.uint32), o32.view(np.uint32))
+
+
+@pytest.mark.parametrize("case", range(16))
+def test_bias_updates_random(cuda_device, case):
+    """SMEBU (clamped and linear) for several layers and the sign update, on
+    random loads (dead experts, skew, an empty layer), random starting state
+    and random fp32 hyper-parameters: bias and momentum within 1e-6 relative
+    of the oracle (bit-identical in practice), MaxVio exact, loads reset."""
+    from tests.parity import STATE_RTOL, rel_err
+    rng = np.random.default_rng(8000 + case)
+    dev = cuda_device
+    f32 = lambda v: float(np.float32(v))
+    L, Nr = int(rng.integers(1, 9)), int(rng.integers(1, 257))
+    lam, beta, kappa = f32(10 ** rng.uniform(-5, -2)), f32(rng.uniform(0, 0.99)), f32(rng.uniform(0.5, 4))
+    gamma = f32(10 ** rng.uniform(-4, -2))
+    linear = case % 3 == 0
+    counts = (rng.pareto(1.5, (L, Nr)) * 50).astype(np.int64)
+    counts[:, rng.choice(Nr, Nr // 10, replace=False)] = 0                 # dead experts
+    if case % 5 == 1:
+        counts[0] = 0                                                     # an empty layer
+    b0 = (rng.standard_normal((L, Nr)) * 0.1).astype(np.float32)
+    m0 = (rng.standard_normal((L, Nr)) * 1e-3).astype(np.float32)
+    c_d = torch.from_numpy(counts.astype(np.int32)).to(dev)
+    b_d, m_d = torch.from_numpy(b0.copy()).to(dev), torch.from_numpy(m0.copy()).to(dev)
+    mv = torch.zeros(L, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ebl.smebu_step_layers(c_d, b_d, m_d, lam, beta, kappa, linear=linear, reset_counts=True, maxvio=mv, status=st)
+    torch.cuda.synchronize()
+    empty = False
+    for l in range(L):
+        b, m = b0[l].copy(), m0[l].copy()
+        if linear:
+            rc, mvo = oracle.smebu_linear(counts[l], b, m, lam, beta)
+        else:
+            rc, mvo = oracle.smebu(counts[l], b, m, lam, beta, kappa)
+        empty |= rc != 0
+        assert rel_err(to_np(b_d[l]), b).max() <= STATE_RTOL, l
+        assert rel_err(to_np(m_d[l]), m).max() <= STATE_RTOL, l
+        assert np.float32(mvo).tobytes() == to_np(mv[l:l + 1]).tobytes(), (l, mvo, float(mv[l]))
+    assert bool(int(st.item()) & ebl.EBL_ST_EMPTY_LOAD) == empty
+    assert int(c_d.abs().sum().item()) == 0
+    # the sign update of the smaller models, on layer L-1's loads
+    c1 = torch.from_numpy(counts[-1].astype(np.int32)).to(dev)
+    b1 = torch.from_numpy(b0[-1].copy()).to(dev)
+    mv1 = torch.zeros(1, device=dev)
+    ebl.sign_update_step(c1, b1, gamma, maxvio=mv1)
+    torch.cuda.synchronize()
+    b = b0[-1].copy()
+    rc, mvo = oracle.sign_update(counts[-1], b, gamma)
+    assert rel_err(to_np(b1), b).max() <= STATE_RTOL
+    assert np.float32(mvo).tobytes() == to_np(mv1).tobytes()
