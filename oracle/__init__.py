@@ -13,6 +13,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+from typing import NamedTuple
 
 import numpy as np
 
@@ -71,6 +72,12 @@ def _bind(path):
     lib.orc_gather_rows.restype = None
     lib.orc_combine.argtypes = [P, P, P, i64, i32, i32, i64, P, P]
     lib.orc_combine.restype = i32
+    lib.orc_seq_balance.argtypes = [P, P, i64, i32, i32, i64, ctypes.c_double, P, P, P, P]
+    lib.orc_seq_balance.restype = i32
+    lib.orc_tile_psum.argtypes = [P, i64, i32, i32, P]
+    lib.orc_tile_psum.restype = i32
+    lib.orc_seq_balance_tiles.argtypes = [P, P, i64, i32, i32, i64, i32, ctypes.c_double, P, P]
+    lib.orc_seq_balance_tiles.restype = i32
     return lib
 
 
@@ -254,3 +261,54 @@ def combine(Y, gates, dest, want64=True, want32=True):
     if rc != ORC_OK:
         raise ValueError("orc_combine returned %d" % rc)
     return o64, o32
+
+
+class SeqBalance(NamedTuple):
+    loss: float             # mean over the sequences of the batch
+    loss_seq: np.ndarray    # fp64 [B]
+    f: np.ndarray           # fp64 [B, N_r]
+    P: np.ndarray           # fp64 [B, N_r]
+
+
+def seq_balance(scores, idx, seq_len, alpha=5e-5):
+    """Sequence-wise balance loss from the router's sigmoid scores [T,N_r]
+    and selections [T,K] (sequences of seq_len consecutive tokens)."""
+    s = _c(scores, np.float64)
+    i = _c(idx, np.int32)
+    T, Nr = s.shape
+    K = i.shape[1]
+    B = T // seq_len if seq_len > 0 else 0
+    f = np.zeros((max(B, 1), Nr))
+    P = np.zeros((max(B, 1), Nr))
+    ls = np.zeros(max(B, 1))
+    loss = np.zeros(1)
+    rc = _load().orc_seq_balance(_ptr(s), _ptr(i), T, Nr, K, seq_len, alpha, _ptr(f), _ptr(P), _ptr(ls), _ptr(loss))
+    if rc != 0:
+        raise ValueError("orc_seq_balance returned %d" % rc)
+    return SeqBalance(float(loss[0]), ls, f, P)
+
+
+def tile_psum(scores, tile_tokens=128):
+    """Per-tile sums of the normalised scores s / sum_j s: fp64 [ceil(T/tile), N_r]."""
+    s = _c(scores, np.float64)
+    T, Nr = s.shape
+    out = np.zeros(((T + tile_tokens - 1) // tile_tokens, Nr))
+    rc = _load().orc_tile_psum(_ptr(s), T, Nr, tile_tokens, _ptr(out))
+    if rc != 0:
+        raise ValueError("orc_tile_psum returned %d" % rc)
+    return out
+
+
+def seq_balance_tiles(tile_counts, psum, T, K, seq_len, alpha=5e-5, tile_tokens=128):
+    """The same loss from per-tile loads and per-tile normalised-score sums.
+    Returns (loss, loss_seq fp64 [B])."""
+    c = _c(tile_counts, np.int32)
+    q = _c(psum, np.float64)
+    Nr = c.shape[1]
+    B = T // seq_len if seq_len > 0 else 0
+    ls = np.zeros(max(B, 1))
+    loss = np.zeros(1)
+    rc = _load().orc_seq_balance_tiles(_ptr(c), _ptr(q), T, Nr, K, seq_len, tile_tokens, alpha, _ptr(ls), _ptr(loss))
+    if rc != 0:
+        raise ValueError("orc_seq_balance_tiles returned %d" % rc)
+    return float(loss[0]), ls

@@ -38,7 +38,11 @@
  *   - gates are g = s / (sum of s over the selected experts), scale 1;
  *   - a "load" n_i counts (token, slot) assignments, so sum n = K*T;
  *   - the sign update re-centres b after adding the step;
- *   - MaxVio is +inf when some expert received no load.
+ *   - MaxVio is +inf when some expert received no load;
+ *   - the sequence-wise balance loss, which the pages name but do not print,
+ *     is the complementary sequence-wise loss of auxiliary-loss-free
+ *     balancing (four equations, as the pages' numbering (29)-(32) suggests),
+ *     averaged over the sequences of a batch.
  */
 #include <math.h>
 #include <stdint.h>
@@ -236,6 +240,116 @@ double orc_router_zloss(const uint16_t *hidden, const uint16_t *W, int64_t T, in
     }
     free(x);
     return total;
+}
+
+/*
+ * Sequence-wise balance loss, the small auxiliary term kept beside the bias
+ * balancing.  [SN] "How it works" names it (eqs. (29)-(32), coefficient
+ * alpha, 5e-5 on the Large checkpoint) and calls it a within-sequence nudge;
+ * [TALK]'s stabilization table describes it as auxiliary load balancing
+ * evaluated per sequence.  The pages do not print the four equations.
+ * Reading: the complementary sequence-wise balance loss published with
+ * auxiliary-loss-free balancing (DeepSeek-V3 technical report, section
+ * 2.1.2), whose four equations are, for one sequence of S tokens:
+ *   f_i    = N_r / (K * S) * #{(t,k) in the sequence : idx_{t,k} = i}
+ *   s'_t,i = s_t,i / sum_j s_t,j        (all N_r experts, no bias)
+ *   P_i    = (1 / S) * sum_t s'_t,i
+ *   L      = alpha * sum_i f_i * P_i
+ * A batch of T tokens holds T / S consecutive sequences; its value is the
+ * mean of their L.
+ * scores: fp64 [T,Nr], the sigmoid scores of the router step; idx: int32
+ * [T,K].  Optional outputs f [B,Nr], P [B,Nr], loss_seq [B]; *loss the mean.
+ */
+int orc_seq_balance(const double *scores, const int32_t *idx, int64_t T, int Nr, int K, int64_t S,
+                    double alpha, double *f_out, double *p_out, double *loss_seq, double *loss)
+{
+    if (T <= 0 || Nr <= 0 || K <= 0 || K > Nr || S <= 0 || T % S != 0) return ORC_EINVAL;
+    for (int64_t p = 0; p < T * K; ++p)
+        if (idx[p] < 0 || idx[p] >= Nr) return ORC_EDATA;
+    const int64_t B = T / S;
+    double *f = (double *)malloc(sizeof(double) * (size_t)Nr);
+    double *P = (double *)malloc(sizeof(double) * (size_t)Nr);
+    double total = 0.0;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int i = 0; i < Nr; ++i) {
+            f[i] = 0.0;
+            P[i] = 0.0;
+        }
+        for (int64_t t = b * S; t < (b + 1) * S; ++t) {
+            for (int k = 0; k < K; ++k) f[idx[t * K + k]] += 1.0;
+            const double *s = scores + t * Nr;
+            double row = 0.0;
+            for (int j = 0; j < Nr; ++j) row += s[j];
+            for (int i = 0; i < Nr; ++i) P[i] += s[i] / row;
+        }
+        double l = 0.0;
+        for (int i = 0; i < Nr; ++i) {
+            f[i] *= (double)Nr / ((double)K * (double)S);
+            P[i] /= (double)S;
+            l += f[i] * P[i];
+        }
+        l *= alpha;
+        if (f_out) memcpy(f_out + b * Nr, f, sizeof(double) * (size_t)Nr);
+        if (p_out) memcpy(p_out + b * Nr, P, sizeof(double) * (size_t)Nr);
+        if (loss_seq) loss_seq[b] = l;
+        total += l;
+    }
+    free(f);
+    free(P);
+    *loss = total / (double)B;
+    return ORC_OK;
+}
+
+/*
+ * The per-tile pieces of the same loss, for tiles of `tile` consecutive tokens
+ * (the last one ragged): psum[j,i] = sum over the tile's tokens t of
+ * s_t,i / sum_l s_t,l.
+ */
+int orc_tile_psum(const double *scores, int64_t T, int Nr, int tile, double *psum)
+{
+    if (T < 0 || Nr <= 0 || tile <= 0) return ORC_EINVAL;
+    const int64_t tiles = (T + tile - 1) / tile;
+    memset(psum, 0, sizeof(double) * (size_t)(tiles * Nr));
+    for (int64_t t = 0; t < T; ++t) {
+        const double *s = scores + t * Nr;
+        double row = 0.0;
+        for (int l = 0; l < Nr; ++l) row += s[l];
+        for (int i = 0; i < Nr; ++i) psum[(t / tile) * Nr + i] += s[i] / row;
+    }
+    return ORC_OK;
+}
+
+/*
+ * The loss from per-tile loads and per-tile sums of normalised scores
+ * (tile_counts [T/tile, Nr] as the router writes them, psum as above), with
+ * S a multiple of tile: the same f_i, P_i and L as orc_seq_balance, each
+ * sequence's loads and sums gathered from its S / tile tiles.
+ */
+int orc_seq_balance_tiles(const int32_t *tile_counts, const double *psum, int64_t T, int Nr, int K, int64_t S,
+                          int tile, double alpha, double *loss_seq, double *loss)
+{
+    if (T <= 0 || Nr <= 0 || K <= 0 || K > Nr || S <= 0 || tile <= 0 || T % S != 0 || S % tile != 0)
+        return ORC_EINVAL;
+    const int64_t B = T / S, per = S / tile;
+    double total = 0.0;
+    for (int64_t b = 0; b < B; ++b) {
+        double l = 0.0;
+        for (int i = 0; i < Nr; ++i) {
+            double n = 0.0, q = 0.0;
+            for (int64_t j = b * per; j < (b + 1) * per; ++j) {
+                n += (double)tile_counts[j * Nr + i];
+                q += psum[j * Nr + i];
+            }
+            const double fi = (double)Nr / ((double)K * (double)S) * n;
+            const double Pi = q / (double)S;
+            l += fi * Pi;
+        }
+        l *= alpha;
+        if (loss_seq) loss_seq[b] = l;
+        total += l;
+    }
+    *loss = total / (double)B;
+    return ORC_OK;
 }
 
 /*

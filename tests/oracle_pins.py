@@ -25,6 +25,11 @@ What pins what:
   - Dispatch: numpy stable argsort; permutation and offset invariants.
   - Combine: numpy einsum in fp64; the identity-expert round trip; the fp32
     chain within its rounding bound.
+  - Sequence-wise balance loss: two hand-derived examples
+    (golden/seq_balance.txt); equal scores give exactly alpha; sum_i P_i = 1
+    and sum_i f_i = N_r per sequence; f from a numpy histogram; invariance
+    under a repeated batch and under shuffles inside a sequence; the per-tile
+    pieces add up to the per-sequence values.
 """
 from __future__ import annotations
 
@@ -511,5 +516,76 @@ def pin_combine_library_and_roundtrip():
     assert np.allclose(r64, hd, rtol=(K + 1) * F32_EPS, atol=0)
     assert np.allclose(r32, hd, rtol=(2 * K + 1) * F32_EPS, atol=0)
 
+
+
+# ------------------------------------------------- sequence-wise balance pins
+
+def _frac(v):
+    from fractions import Fraction
+    return float(Fraction(v))
+
+
+def pin_seq_balance_golden():
+    g = _read_kv("seq_balance.txt")
+    for ex in ("A", "B"):
+        T, Nr, K, S = (int(v) for v in g[ex + "_shape"])
+        scores = np.array([_frac(v) for v in g[ex + "_scores"]]).reshape(T, Nr)
+        idx = np.array([int(v) for v in g[ex + "_idx"]], np.int32).reshape(T, K)
+        r = oracle.seq_balance(scores, idx, S, _frac(g[ex + "_alpha"][0]))
+        for key, got in (("f", r.f), ("P", r.P), ("loss_seq", r.loss_seq)):
+            want = np.array([_frac(v) for v in g[ex + "_" + key]])
+            assert np.allclose(got.reshape(-1), want, rtol=1e-14, atol=1e-300), (ex, key, got, want)
+        want = _frac(g[ex + "_loss"][0])
+        assert abs(r.loss - want) <= 1e-14 * want, (ex, r.loss, want)
+
+
+def pin_seq_balance_equal_scores_and_invariants():
+    rng = np.random.default_rng(29)
+    Nr, K, S, B = 16, 3, 64, 6
+    T = B * S
+    idx = np.stack([rng.choice(Nr, K, replace=False) for _ in range(T)]).astype(np.int32)
+    alpha = 5e-5
+    # every score equal: s' = 1/N_r, so P_i = 1/N_r and L = alpha * (sum_i f_i) / N_r = alpha
+    r = oracle.seq_balance(np.full((T, Nr), 0.3), idx, S, alpha)
+    assert np.allclose(r.loss_seq, alpha, rtol=1e-13, atol=0) and abs(r.loss - alpha) <= 1e-13 * alpha
+    scores = expit(rng.standard_normal((T, Nr)) * 2)
+    r = oracle.seq_balance(scores, idx, S, alpha)
+    assert np.allclose(r.P.sum(1), 1.0, rtol=1e-13, atol=0)          # s' sums to 1 per token
+    assert np.allclose(r.f.sum(1), Nr, rtol=1e-13, atol=0)           # K*S selections per sequence
+    for b in range(B):                                               # f from a library histogram
+        n = np.bincount(idx[b * S:(b + 1) * S].reshape(-1), minlength=Nr)
+        assert np.allclose(r.f[b] * (K * S) / Nr, n, rtol=1e-14, atol=1e-14)
+    assert abs(r.loss - r.loss_seq.mean()) <= 1e-15 * r.loss
+    # a batch of the same sequences twice has the same value; a shuffle of the
+    # tokens inside each sequence leaves every sequence's value unchanged
+    r2 = oracle.seq_balance(np.concatenate([scores, scores]), np.concatenate([idx, idx]), S, alpha)
+    assert abs(r2.loss - r.loss) <= 1e-14 * r.loss
+    perm = np.concatenate([b * S + rng.permutation(S) for b in range(B)])
+    r3 = oracle.seq_balance(scores[perm], idx[perm], S, alpha)
+    assert np.allclose(r3.loss_seq, r.loss_seq, rtol=1e-13, atol=0)
+    # all of a sequence on one expert with K = 1: f = N_r there, so L = alpha N_r P_e
+    one = np.zeros((S, 1), np.int32) + 5
+    r4 = oracle.seq_balance(scores[:S], one, S, alpha)
+    assert abs(r4.loss - alpha * Nr * r4.P[0, 5]) <= 1e-14 * r4.loss
+
+
+def pin_seq_balance_tiles_agree():
+    rng = np.random.default_rng(31)
+    Nr, K, S, B, tile = 24, 2, 256, 3, 128
+    T = B * S
+    idx = np.stack([rng.choice(Nr, K, replace=False) for _ in range(T)]).astype(np.int32)
+    scores = expit(rng.standard_normal((T, Nr)))
+    psum = oracle.tile_psum(scores, tile)
+    assert np.allclose(psum.sum(1), tile, rtol=1e-13, atol=0)       # one unit of s' per token
+    rag = oracle.tile_psum(scores[:T - 37], tile)
+    assert rag.shape[0] == T // tile and abs(rag[-1].sum() - (tile - 37)) <= 1e-12
+    counts = np.stack([np.bincount(idx[j * tile:(j + 1) * tile].reshape(-1), minlength=Nr)
+                       for j in range(T // tile)]).astype(np.int32)
+    ref = oracle.seq_balance(scores, idx, S, 5e-5)
+    loss, loss_seq = oracle.seq_balance_tiles(counts, psum, T, K, S, 5e-5, tile)
+    assert np.allclose(loss_seq, ref.loss_seq, rtol=1e-12, atol=0) and abs(loss - ref.loss) <= 1e-12 * ref.loss
+    per = S // tile
+    for b in range(B):
+        assert np.allclose(psum[b * per:(b + 1) * per].sum(0), S * ref.P[b], rtol=1e-12, atol=0)
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -61,6 +61,18 @@ MUTANTS = {
                  "gap_out[t] = (K == Nr) ? INFINITY : best_rest - key[sel[K - 1]];"),
     "gap_from_first_slot": ("gap_out[t] = (K == Nr) ? INFINITY : key[sel[K - 1]] - best_rest;",
                             "gap_out[t] = (K == Nr) ? INFINITY : key[sel[0]] - best_rest;"),
+    "seqbal_unnormalised": ("for (int i = 0; i < Nr; ++i) P[i] += s[i] / row;",
+                            "for (int i = 0; i < Nr; ++i) P[i] += s[i];"),
+    "seqbal_no_nr_factor": ("f[i] *= (double)Nr / ((double)K * (double)S);",
+                            "f[i] *= 1.0 / ((double)K * (double)S);"),
+    "seqbal_no_k": ("f[i] *= (double)Nr / ((double)K * (double)S);", "f[i] *= (double)Nr / (double)S;"),
+    "seqbal_p_not_averaged": ("            P[i] /= (double)S;\n", ""),
+    "seqbal_sum_not_mean": ("    free(P);\n    *loss = total / (double)B;", "    free(P);\n    *loss = total;"),
+    "seqbal_gates_as_s_prime": ("for (int j = 0; j < Nr; ++j) row += s[j];",
+                                "for (int j = 0; j < K; ++j) row += s[idx[t * K + j]];"),
+    "tile_psum_unnormalised": ("psum[(t / tile) * Nr + i] += s[i] / row;", "psum[(t / tile) * Nr + i] += s[i];"),
+    "seqbal_tiles_first_sequence": ("for (int64_t j = b * per; j < (b + 1) * per; ++j) {",
+                                    "for (int64_t j = 0; j < per; ++j) {"),
     "combine_drops_slot": ("            for (int k = 0; k < K; ++k) {\n                const int64_t row",
                            "            for (int k = 0; k < K - 1; ++k) {\n                const int64_t row"),
 }
