@@ -420,6 +420,32 @@ def main():
         torch.cuda.synchronize()
         extra["zloss_router_ms"] = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
         del zl
+        # the balance option (per-tile statistics of the sequence-wise balance
+        # loss) and the loss itself, sequences of 4096 tokens
+        seq_len = 4096 if T % 4096 == 0 else 128 * (T // 128) if T % 128 == 0 else 0
+        if seq_len:
+            tcb = torch.empty((T + 127) // 128, Nr, dtype=torch.int32, device=dev)
+            tpb = torch.empty((T + 127) // 128, Nr, dtype=torch.float32, device=dev)
+            lseq = torch.empty(T // seq_len, dtype=torch.float64, device=dev)
+            lval = torch.empty(1, dtype=torch.float64, device=dev)
+
+            def balance_step():
+                ebl.router_forward_balance(h, W, bias, K, counts, tcb, tpb, topk_idx=idx, gates=gates, stream=stream)
+                ebl.seq_balance_loss(tcb, tpb, T, K, seq_len, loss_seq=lseq, loss=lval, stream=stream)
+
+            for _ in range(2):
+                balance_step()
+            counts.zero_()
+            ev[0].record(stream)
+            for _ in range(reps):
+                balance_step()
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            bm = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
+            extra["seq_balance"] = {"seq_len": seq_len, "router_balance_and_loss_ms": bm,
+                                    "tokens_per_s": T * world / (bm / 1e3)}
+            counts.zero_()
+            del tcb, tpb, lseq, lval
         x = synth.logits_normal(T, Nr, seed=synth.step_seed(WORKLOAD, 1) + 1000 * rank, device=dev, quant8=True)
         for _ in range(2):
             ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=gates, stream=stream)

@@ -21,11 +21,12 @@ import os
 import torch
 
 __all__ = [
-    "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_logits", "smebu_step",
+    "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_balance",
+    "seq_balance_loss", "router_forward_logits", "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
     "read_internal_status", "check_finite", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD",
     "EBL_ST_TIMEOUT", "EBL_ST_BAD_COUNTS", "EBL_ST_NONFINITE",
-    "SMEBU_LAMBDA", "SMEBU_BETA", "SMEBU_KAPPA",
+    "SMEBU_LAMBDA", "SMEBU_BETA", "SMEBU_KAPPA", "SEQ_BALANCE_ALPHA",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +38,9 @@ EBL_ST_NONFINITE = 32
 
 # Trinity Large's SMEBU constants ("Arcee Trinity Large Technical Report" 2.3)
 SMEBU_LAMBDA, SMEBU_BETA, SMEBU_KAPPA = 5e-4, 0.5, 2.0
+# coefficient of the sequence-wise balance loss on the Large checkpoint
+# ("SMEBU Load Balancing", "How it works")
+SEQ_BALANCE_ALPHA = 5e-5
 
 # exported symbol -> (restype, argtypes); the full C ABI of include/ebl.h
 _P = ctypes.c_void_p
@@ -51,6 +55,8 @@ SIGNATURES = {
     "router_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "router_forward_zloss": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "router_forward_logits": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "router_forward_balance": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "seq_balance_loss": (_I, [_P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "smebu_step": (_I, [_P, _P, _P, _I, _F, _F, _F, _I, _P, _P, _P]),
     "smebu_step_layers": (_I, [_P, _P, _P, _I, _I, _F, _F, _F, _I, _I, _P, _P, _P]),
     "sign_update_step": (_I, [_P, _P, _I, _F, _I, _P, _P, _P]),
@@ -185,6 +191,51 @@ def router_forward_zloss(hidden, W_router, bias, K, counts, zloss_sum, topk_idx=
     _call("router_forward_zloss", _ptr(hidden), _ptr(W_router), _ptr(bias), T, d, Nr, K, _ptr(topk_idx),
           _ptr(gates), _ptr(counts), _ptr(tile_counts), _ptr(zloss_sum), _ptr(status), _stream(stream))
     return topk_idx, gates
+
+
+def router_forward_balance(hidden, W_router, bias, K, counts, tile_counts, tile_psum, zloss_sum=None, topk_idx=None,
+                           gates=None, status=None, stream=None):
+    """router_forward that also writes the per-tile statistics of the
+    sequence-wise balance loss: tile_counts int32 and tile_psum fp32, both
+    [ceil(T/128), N_r] (sums of s / sum_j s over each tile's tokens); with
+    zloss_sum (fp64 [1]) it accumulates the z-loss statistic too.
+    Returns (topk_idx, gates)."""
+    _check(hidden, "hidden", torch.bfloat16)
+    T, d = hidden.shape
+    Nr = W_router.shape[0]
+    _check(W_router, "W_router", torch.bfloat16, (Nr, d))
+    _check(bias, "bias", torch.float32, (Nr,))
+    _check(counts, "counts", torch.int32, (Nr,))
+    tiles = (T + 127) // 128
+    _check(tile_counts, "tile_counts", torch.int32, (tiles, Nr))
+    _check(tile_psum, "tile_psum", torch.float32, (tiles, Nr))
+    if zloss_sum is not None:
+        _check(zloss_sum, "zloss_sum", torch.float64, (1,))
+    dev = hidden.device
+    topk_idx = _out(topk_idx, "topk_idx", (T, K), torch.int32, dev)
+    gates = _out(gates, "gates", (T, K), torch.float32, dev)
+    _call("router_forward_balance", _ptr(hidden), _ptr(W_router), _ptr(bias), T, d, Nr, K, _ptr(topk_idx),
+          _ptr(gates), _ptr(counts), _ptr(tile_counts), _ptr(tile_psum), _ptr(zloss_sum), _ptr(status),
+          _stream(stream))
+    return topk_idx, gates
+
+
+def seq_balance_loss(tile_counts, tile_psum, T, K, seq_len, alpha=SEQ_BALANCE_ALPHA, loss_seq=None, loss=None,
+                     stream=None):
+    """Sequence-wise balance loss from router_forward_balance's per-tile
+    statistics (sequences of seq_len consecutive tokens, seq_len % 128 == 0,
+    T % seq_len == 0).  Returns (loss fp64 [1], loss_seq fp64 [T/seq_len])."""
+    tiles = (T + 127) // 128
+    Nr = tile_counts.shape[1]
+    _check(tile_counts, "tile_counts", torch.int32, (tiles, Nr))
+    _check(tile_psum, "tile_psum", torch.float32, (tiles, Nr))
+    dev = tile_counts.device
+    B = T // seq_len if seq_len > 0 else 0
+    loss_seq = _out(loss_seq, "loss_seq", (B,), torch.float64, dev)
+    loss = _out(loss, "loss", (1,), torch.float64, dev)
+    _call("seq_balance_loss", _ptr(tile_counts), _ptr(tile_psum), T, Nr, K, seq_len, alpha, _ptr(loss_seq),
+          _ptr(loss), _stream(stream))
+    return loss, loss_seq
 
 
 def router_forward_logits(logits, bias, K, counts, topk_idx=None, gates=None, tile_counts=None, status=None,

@@ -117,7 +117,7 @@ namespace {
 
 int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d, int N_r,
                      int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
-                     double *zloss_sum, int32_t *status, ebl_stream_t stream) {
+                     double *zloss_sum, float *tile_psum, int32_t *status, ebl_stream_t stream) {
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
     if (d < 64 || d > (1 << 20) || d % 64 != 0) return EBL_EINVAL;
     if (N_r % 32 != 0) return EBL_EUNSUPPORTED;
@@ -127,6 +127,7 @@ int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const flo
     if (K % 4 == 0 && (!aligned16(topk_idx) || !aligned16(gates))) return EBL_EINVAL;
     if (!aligned4(topk_idx) || !aligned4(gates) || (tile_counts && !aligned4(tile_counts))) return EBL_EINVAL;
     if (zloss_sum && (reinterpret_cast<uintptr_t>(zloss_sum) & 7u)) return EBL_EINVAL;
+    if (tile_psum && (!aligned4(tile_psum) || (T > 0 && !tile_counts))) return EBL_EINVAL;
     if (T == 0) return EBL_OK;
     DeviceInfo di;
     int rc = device_info(&di);
@@ -137,7 +138,7 @@ int router_gemm_call(const uint16_t *hidden, const uint16_t *W_router, const flo
     if ((rc = encode_bf16_2d(&tw, W_router, (uint64_t)N_r, (uint64_t)d, (uint32_t)ebl::router_gemm_w_box_rows(N_r))))
         return rc;
     cudaError_t e = ebl::launch_router_gemm(th, tw, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts,
-                                            zloss_sum, status ? status : di.internal_status, di.num_sms,
+                                            zloss_sum, tile_psum, status ? status : di.internal_status, di.num_sms,
                                             reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
@@ -173,7 +174,7 @@ int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float
                    int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
                    ebl_stream_t stream) {
     return router_gemm_call(hidden, W_router, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts, nullptr,
-                            status, stream);
+                            nullptr, status, stream);
 }
 
 int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d,
@@ -181,7 +182,29 @@ int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const
                          double *zloss_sum, int32_t *status, ebl_stream_t stream) {
     if (!zloss_sum) return EBL_EINVAL;
     return router_gemm_call(hidden, W_router, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts, zloss_sum,
-                            status, stream);
+                            nullptr, status, stream);
+}
+
+int router_forward_balance(const uint16_t *hidden, const uint16_t *W_router, const float *bias, int T, int d,
+                           int N_r, int K, int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                           float *tile_psum, double *zloss_sum, int32_t *status, ebl_stream_t stream) {
+    if (T > 0 && (!tile_counts || !tile_psum)) return EBL_EINVAL;
+    return router_gemm_call(hidden, W_router, bias, T, d, N_r, K, topk_idx, gates, counts, tile_counts, zloss_sum,
+                            tile_psum, status, stream);
+}
+
+int seq_balance_loss(const int32_t *tile_counts, const float *tile_psum, int T, int N_r, int K, int seq_len,
+                     float alpha, double *loss_seq, double *loss, ebl_stream_t stream) {
+    if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
+    if (seq_len <= 0 || seq_len % ebl::kTileTokens != 0 || T % seq_len != 0) return EBL_EINVAL;
+    if (!(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return EBL_EINVAL;  // NaN or infinite
+    if (T == 0) return EBL_OK;
+    if (!tile_counts || !tile_psum || !loss_seq || !loss) return EBL_EINVAL;
+    if (!aligned4(tile_counts) || !aligned4(tile_psum)) return EBL_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(loss_seq) & 7u) || (reinterpret_cast<uintptr_t>(loss) & 7u)) return EBL_EINVAL;
+    cudaError_t e = ebl::launch_seq_balance(tile_counts, tile_psum, T, N_r, K, seq_len, alpha, loss_seq, loss,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 
 int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K, int32_t *topk_idx,

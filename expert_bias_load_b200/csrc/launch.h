@@ -18,8 +18,8 @@ constexpr int kMaxTopK = 8;       // K limit
 int router_gemm_w_box_rows(int Nr);  // rows of W per TMA box (N_r / CTAs per MMA)
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
-                               int32_t *tile_counts, double *zloss_sum, int32_t *status, int num_sms,
-                               cudaStream_t stream);
+                               int32_t *tile_counts, double *zloss_sum, float *tile_psum, int32_t *status,
+                               int num_sms, cudaStream_t stream);
 
 // router_logits.cu
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
@@ -36,6 +36,10 @@ cudaError_t launch_smebu(int32_t *counts, float *bias, float *momentum, int L, i
                          cudaStream_t stream);
 cudaError_t launch_sign_update(int32_t *counts, float *bias, int Nr, float gamma, int reset_counts,
                                float *maxvio_out, int32_t *status, cudaStream_t stream);
+
+// seq_balance.cu
+cudaError_t launch_seq_balance(const int32_t *tile_counts, const float *tile_psum, int T, int Nr, int K, int seq_len,
+                               float alpha, double *loss_seq, double *loss, cudaStream_t stream);
 
 // dispatch.cu
 size_t dispatch_workspace_bytes(int T, int Nr);

@@ -30,6 +30,12 @@
 //               gates, and keeps the load histogram (and, for the z-loss, a
 //               running log-sum-exp per row).  Two epilogue warps per SM
 //               sub-partition keep up with the MMAs.
+//   balance     optionally (for the sequence-wise balance loss) each thread
+//               also totals its row's scores; the groups exchange the totals,
+//               read the accumulator a second time, and fold the normalised
+//               scores s / total of their 32 rows into column sums with warp
+//               shuffles; the tile's sums per expert go to tile_psum in a
+//               fixed order, so they are deterministic.
 // The logits never leave TMEM.  Counts reach global memory with one atomic per
 // expert per CTA; tile_counts with one store per expert per tile.  Every
 // pipeline wait is bounded (EBL_ST_TIMEOUT, then a clean exit).
@@ -66,13 +72,20 @@ __host__ __device__ inline uint32_t tmem_columns(int Nr) {
     return c;
 }
 
+// Kernel options (the E template argument): z-loss statistic, and the
+// per-tile statistics of the sequence-wise balance loss.
+constexpr int kOptZloss = 1;
+constexpr int kOptBalance = 2;
+
 // Shared memory after the stage ring: barriers, then (16-byte aligned) the
-// bias, the histograms and the partial-list exchange buffers.
+// bias, the histograms and the partial-list exchange buffers; with the balance
+// option, two more barriers, the per-row score totals of every group and the
+// per-warp column sums.
 struct Misc {
-    size_t bar_off, vec_off, total;
+    size_t bar_off, vec_off, aux_off, total;
 };
 
-__host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int stages) {
+__host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int stages, int E) {
     Misc m;
     m.bar_off = (size_t)stages * (kATileBytes + b_tile_bytes(Nr));
     // full[S], empty[S], tfull[2], tempty[2], epi_sync, drain, list_full, list_empty; tmem slot, abort flag
@@ -80,7 +93,9 @@ __host__ __device__ inline Misc misc_layout(int Nr, int K, int G, int stages) {
     m.vec_off = m.bar_off + ((bars + 15) & ~size_t(15));
     const size_t vec = (size_t)4 * Nr * 4 + (size_t)3 * (G - 1) * K * kTileTokens * 4 +
                        (size_t)2 * (G - 1) * kTileTokens * 4;  // partial lists; partial log-sum-exp
-    m.total = m.vec_off + vec;
+    m.aux_off = (m.vec_off + vec + 15) & ~size_t(15);
+    m.total = m.aux_off;
+    if (E & kOptBalance) m.total += 16 + (size_t)(G * kTileTokens + 4 * Nr) * 4;
     return m;
 }
 
@@ -105,9 +120,9 @@ struct RowLse {
     }
 };
 
-template <int K, bool Z>
+template <int K, bool Z, bool P>
 __device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const float *__restrict__ bias_s, int c,
-                                              RowTopK<K> &tk, RowLse &lse) {
+                                              RowTopK<K> &tk, RowLse &lse, float &rsum) {
     if constexpr (Z) {  // z-loss: log-sum-exp of the chunk, folded into the row's
         float cm = __uint_as_float(r[0]);
 #pragma unroll
@@ -126,25 +141,62 @@ __device__ __forceinline__ void consume_chunk(const uint32_t (&r)[kChunk], const
         for (int j = 0; j < 4; ++j) {
             const float x = __uint_as_float(r[4 * q + j]);
             const float s = fast_rcp(1.0f + __expf(-x));
+            if constexpr (P) rsum += s;
             tk.push(__fadd_rn(s, bv[j]), s, c + 4 * q + j);
         }
     }
 }
 
-template <int K, int G, bool Z>
+// One step of a warp's column sums over its 32 rows: each lane keeps W of its
+// 2W values, the half picked by lane bit 2W, and adds the partner's matching
+// half (partner = lane ^ 2W).
+template <int W>
+__device__ __forceinline__ void column_fold(float (&v)[kChunk], int lane) {
+    const bool hi = (lane & (2 * W)) != 0;
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+        const float send = hi ? v[j] : v[j + W];
+        const float keep = hi ? v[j + W] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2 * W);
+    }
+}
+
+// Sums over the warp's 32 rows of the 16 columns in v (this lane's row):
+// lanes 2c and 2c + 1 return the sum of column c.  31 shuffles per 16 columns.
+__device__ __forceinline__ float warp_column_sums(float (&v)[kChunk], int lane) {
+    column_fold<8>(v, lane);
+    column_fold<4>(v, lane);
+    column_fold<2>(v, lane);
+    column_fold<1>(v, lane);
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// Normalised scores s / total of one 16-column chunk (inv = 1 / total, or 0
+// for a row past T), folded into the warp's column sums and stored in pw.
+__device__ __forceinline__ void balance_chunk(const uint32_t (&r)[kChunk], float inv, int lane, float *pw) {
+    float v[kChunk];
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) v[j] = fast_rcp(1.0f + __expf(-__uint_as_float(r[j]))) * inv;
+    const float sum = warp_column_sums(v, lane);
+    if ((lane & 1) == 0) pw[lane >> 1] = sum;
+}
+
+template <int K, int G, int E>
 __global__ void __launch_bounds__(threads_of(G), 1)
     router_gemm_kernel(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
                        const float *__restrict__ bias, int T, int d, int Nr, int stages,
                        int32_t *__restrict__ topk_idx, float *__restrict__ gates, int32_t *__restrict__ counts,
                        int32_t *__restrict__ tile_counts, double *__restrict__ zloss_sum,
-                       int32_t *__restrict__ status) {
+                       float *__restrict__ tile_psum, int32_t *__restrict__ status) {
+    constexpr bool Z = (E & kOptZloss) != 0;
+    constexpr bool P = (E & kOptBalance) != 0;
     constexpr int kEpiWarps = 4 * G;
     constexpr int kProducerWarp = 4 * G;
     constexpr int kMmaWarp = 4 * G + 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-    const Misc ml = misc_layout(Nr, K, G, stages);
+    const Misc ml = misc_layout(Nr, K, G, stages, E);
     const uint32_t b_bytes = b_tile_bytes(Nr);
     uint8_t *smA = smem;
     uint8_t *smB = smem + (size_t)stages * kATileBytes;
@@ -166,6 +218,10 @@ __global__ void __launch_bounds__(threads_of(G), 1)
     int *pl_idx = reinterpret_cast<int *>(pl_s + (G - 1) * K * kTileTokens);
     float *pl_zm = reinterpret_cast<float *>(pl_idx + (G - 1) * K * kTileTokens);  // [G-1][128]
     float *pl_zs = pl_zm + (G - 1) * kTileTokens;
+    uint64_t *rows_ready = reinterpret_cast<uint64_t *>(smem + ml.aux_off);  // balance option only
+    uint64_t *cols_ready = rows_ready + 1;
+    float *row_total = reinterpret_cast<float *>(cols_ready + 1);  // [G][128]
+    float *col_part = row_total + G * kTileTokens;                 // [4][Nr]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -198,6 +254,10 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         mbar_init(drain, 1);
         mbar_init(list_full, (G - 1) * 128 > 0 ? (G - 1) * 128 : 1);
         mbar_init(list_empty, 128);
+        if constexpr (P) {
+            mbar_init(rows_ready, kEpiWarps * 32);
+            mbar_init(cols_ready, kEpiWarps * 32);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmap_h);
@@ -313,7 +373,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
         const int c0 = group * cpg;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         const bool want_tiles = tile_counts != nullptr;
-        uint32_t sync_ph = 0;
+        uint32_t sync_ph = 0, aux_ph = 0;
         bool ok = true;
         int it = 0;
         float zacc = 0.0f;  // this thread's rows: sum of log-sum-exp squared
@@ -331,6 +391,7 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             tk.init();
             RowLse lse;
             lse.init();
+            float rsum = 0.0f;
             const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * Nr + c0);
             uint32_t ra[kChunk], rb[kChunk];
             __syncwarp();
@@ -339,19 +400,62 @@ __global__ void __launch_bounds__(threads_of(G), 1)
             for (int c = 0; c < cpg; c += 2 * kChunk) {  // cpg % 32 == 0: chunks come in pairs
                 __syncwarp();
                 tmem_ld_32x32b_x16(taddr + (uint32_t)(c + kChunk), rb);
-                consume_chunk<K, Z>(ra, bias_s, c0 + c, tk, lse);
+                consume_chunk<K, Z, P>(ra, bias_s, c0 + c, tk, lse, rsum);
                 __syncwarp();
                 tmem_ld_wait_x16(rb);
                 const bool more = c + 2 * kChunk < cpg;
                 if (more) tmem_ld_32x32b_x16(taddr + (uint32_t)(c + 2 * kChunk), ra);
-                consume_chunk<K, Z>(rb, bias_s, c0 + c + kChunk, tk, lse);
+                consume_chunk<K, Z, P>(rb, bias_s, c0 + c + kChunk, tk, lse, rsum);
                 __syncwarp();
                 if (more) tmem_ld_wait_x16(ra);
+            }
+            if constexpr (P) {
+                // the row's total over all experts (groups in order, the same sum
+                // in every group), then a second pass over this group's columns
+                row_total[group * kTileTokens + rloc] = rsum;
+                mbar_arrive(rows_ready);
+                if (!mbar_wait(rows_ready, aux_ph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                float total = 0.0f;
+#pragma unroll
+                for (int g = 0; g < G; ++g) total += row_total[g * kTileTokens + rloc];
+                const float inv = (tile * kTileTokens + rloc < T && total > 0.0f) ? __frcp_rn(total) : 0.0f;
+                float *pw = col_part + quad * Nr + c0;
+                __syncwarp();
+                tmem_ld_32x32b_x16(taddr, ra);
+                tmem_ld_wait_x16(ra);
+                for (int c = 0; c < cpg; c += 2 * kChunk) {
+                    __syncwarp();
+                    tmem_ld_32x32b_x16(taddr + (uint32_t)(c + kChunk), rb);
+                    balance_chunk(ra, inv, lane, pw + c);
+                    __syncwarp();
+                    tmem_ld_wait_x16(rb);
+                    const bool more = c + 2 * kChunk < cpg;
+                    if (more) tmem_ld_32x32b_x16(taddr + (uint32_t)(c + 2 * kChunk), ra);
+                    balance_chunk(rb, inv, lane, pw + c + kChunk);
+                    __syncwarp();
+                    if (more) tmem_ld_wait_x16(ra);
+                }
+                mbar_arrive(cols_ready);
             }
             // this warp is done with the accumulator: hand it back to the MMA warp
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_u32(&tempty[acc]), 0));
+            if constexpr (P) {
+                // the tile's column sums: the four row quadrants in order
+                if (!mbar_wait(cols_ready, aux_ph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                aux_ph ^= 1u;
+                if (tile < num_tiles)
+                    for (int e = (int)threadIdx.x; e < Nr; e += kEpiWarps * 32)
+                        tile_psum[(size_t)tile * Nr + e] =
+                            ((col_part[e] + col_part[Nr + e]) + col_part[2 * Nr + e]) + col_part[3 * Nr + e];
+            }
 
             if (group > 0) {
                 // publish the sorted partial list for group 0
@@ -482,10 +586,10 @@ __global__ void __launch_bounds__(threads_of(G), 1)
 // with the MMAs and leave more issue slots to the TMA and MMA warps than 16.
 int groups_for(int Nr) { return (Nr % 64 == 0) ? 2 : 1; }
 
-int stages_for(int Nr, int K, int G) {  // the layout is the same with and without z-loss
+int stages_for(int Nr, int K, int G, int E) {
     const size_t budget = 232448;  // max dynamic shared memory per CTA on sm_100
     int s = kMaxStages;
-    while (s > 2 && 1024 + misc_layout(Nr, K, G, s).total > budget) --s;
+    while (s > 2 && 1024 + misc_layout(Nr, K, G, s, E).total > budget) --s;
     return s;
 }
 
@@ -543,10 +647,18 @@ cudaError_t launch_setup(const void *kern, size_t smem, cudaLaunchConfig_t *cfg,
 template <int K, int G>
 cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
                       int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zloss_sum,
-                      int32_t *status, int num_sms, cudaStream_t stream) {
-    auto kern = zloss_sum ? router_gemm_kernel<K, G, true> : router_gemm_kernel<K, G, false>;
-    const int stages = stages_for(Nr, K, G);
-    const size_t smem = 1024 + misc_layout(Nr, K, G, stages).total;
+                      float *tile_psum, int32_t *status, int num_sms, cudaStream_t stream) {
+    const int E = (zloss_sum ? kOptZloss : 0) | (tile_psum ? kOptBalance : 0);
+    void (*kern)(CUtensorMap, CUtensorMap, const float *, int, int, int, int, int32_t *, float *, int32_t *,
+                 int32_t *, double *, float *, int32_t *);
+    switch (E) {
+        case kOptZloss: kern = router_gemm_kernel<K, G, kOptZloss>; break;
+        case kOptBalance: kern = router_gemm_kernel<K, G, kOptBalance>; break;
+        case kOptZloss | kOptBalance: kern = router_gemm_kernel<K, G, kOptZloss | kOptBalance>; break;
+        default: kern = router_gemm_kernel<K, G, 0>; break;
+    }
+    const int stages = stages_for(Nr, K, G, E);
+    const size_t smem = 1024 + misc_layout(Nr, K, G, stages, E).total;
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     const int num_work = (num_tiles + kPair - 1) / kPair;
     int units = num_sms / kPair;
@@ -569,20 +681,22 @@ cudaError_t launch_kg(const CUtensorMap &th, const CUtensorMap &tw, const float 
     if (units > num_work) units = num_work;
     cfg.gridDim = dim3(kPair * units, 1, 1);
     err = cudaLaunchKernelEx(&cfg, kern, th, tw, bias, T, d, Nr, stages, idx, gates, counts, tile_counts, zloss_sum,
-                             status);
+                             tile_psum, status);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
 }
 
 template <int K>
 cudaError_t launch_k(const CUtensorMap &th, const CUtensorMap &tw, const float *bias, int T, int d, int Nr,
-                     int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zl,
+                     int32_t *idx, float *gates, int32_t *counts, int32_t *tile_counts, double *zl, float *psum,
                      int32_t *status, int num_sms, cudaStream_t stream) {
     switch (groups_for(Nr)) {
         case 2:
-            return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
+            return launch_kg<K, 2>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, psum, status, num_sms,
+                                   stream);
         default:
-            return launch_kg<K, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, status, num_sms, stream);
+            return launch_kg<K, 1>(th, tw, bias, T, d, Nr, idx, gates, counts, tile_counts, zl, psum, status, num_sms,
+                                   stream);
     }
 }
 
@@ -592,13 +706,13 @@ int router_gemm_w_box_rows(int Nr) { return Nr / kPair; }
 
 cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tmap_w, const float *bias, int T,
                                int d, int Nr, int K, int32_t *topk_idx, float *gates, int32_t *counts,
-                               int32_t *tile_counts, double *zloss_sum, int32_t *status, int num_sms,
-                               cudaStream_t stream) {
+                               int32_t *tile_counts, double *zloss_sum, float *tile_psum, int32_t *status,
+                               int num_sms, cudaStream_t stream) {
     switch (K) {
 #define EBL_CASE(KK) \
     case KK:         \
-        return launch_k<KK>(tmap_h, tmap_w, bias, T, d, Nr, topk_idx, gates, counts, tile_counts, zloss_sum, status, \
-                             num_sms, stream);
+        return launch_k<KK>(tmap_h, tmap_w, bias, T, d, Nr, topk_idx, gates, counts, tile_counts, zloss_sum, \
+                             tile_psum, status, num_sms, stream);
         EBL_CASE(1)
         EBL_CASE(2)
         EBL_CASE(3)

@@ -9,8 +9,10 @@ second, and the bytes or flops per call over that time.  It runs nothing but the
 public binding, so it is also the command to put under a profiler: with
 `--warmup W` the timed calls are launches W+1 ... W+reps of that kernel.
 
-Entry points: router (GEMM mode), zloss (GEMM mode with the z-loss), logits
-(logits mode), smebu, sign, dispatch, combine.  For the one-CTA update kernels
+Entry points: router (GEMM mode), zloss (GEMM mode with the z-loss), balance
+(GEMM mode with the sequence-wise balance statistics, then the loss over
+sequences of 4096 tokens, or of T tokens when T is smaller), logits (logits
+mode), smebu, sign, dispatch, combine.  For the one-CTA update kernels
 (smebu, sign) the time per call is the host's launch rate, not the kernel's.
 """
 from __future__ import annotations
@@ -38,7 +40,7 @@ def _time(fn, warmup, reps):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("op", choices=["router", "zloss", "logits", "smebu", "sign", "dispatch", "combine"])
+    ap.add_argument("op", choices=["router", "zloss", "balance", "logits", "smebu", "sign", "dispatch", "combine"])
     ap.add_argument("--tokens", type=int, default=1 << 20)
     ap.add_argument("--hidden", type=int, default=4096)
     ap.add_argument("--experts", type=int, default=256)
@@ -54,13 +56,23 @@ def main(argv=None):
     bias = synth.dead_start_bias(Nr, device=dev)
     counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
     work = ""
-    if a.op in ("router", "zloss"):
+    if a.op in ("router", "zloss", "balance"):
         h = synth.hidden_normal(T, d, seed=a.seed, device=dev, quant8=True)
         W = synth.router_weight(Nr, d, seed=a.seed + 1).to(dev)
         idx = torch.empty(T, K, dtype=torch.int32, device=dev)
         g = torch.empty(T, K, device=dev)
         if a.op == "router":
             fn = lambda: ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=g)
+        elif a.op == "balance":
+            S = 4096 if T % 4096 == 0 else T
+            if T % 128:
+                raise SystemExit("balance needs --tokens a multiple of 128")
+            tc = torch.empty(T // 128, Nr, dtype=torch.int32, device=dev)
+            tp = torch.empty(T // 128, Nr, device=dev)
+
+            def fn():
+                ebl.router_forward_balance(h, W, bias, K, counts, tc, tp, topk_idx=idx, gates=g)
+                ebl.seq_balance_loss(tc, tp, T, K, S)
         else:
             zl = torch.zeros(1, dtype=torch.float64, device=dev)
             fn = lambda: ebl.router_forward_zloss(h, W, bias, K, counts, zl, topk_idx=idx, gates=g)

@@ -138,6 +138,54 @@ int router_forward_zloss(const uint16_t *hidden, const uint16_t *W_router, const
                          double *zloss_sum, int32_t *status, ebl_stream_t stream);
 
 /*
+ * router_forward_balance -- router_forward that also writes the per-tile
+ * statistics of the sequence-wise balance loss (and, if zloss_sum is not
+ * NULL, accumulates the z-loss statistic as router_forward_zloss does):
+ *   tile_psum[j, i] = sum over tokens t in [128 j, 128 j + 128), t < T, of
+ *                     s_{t,i} / sum_l s_{t,l}       (all N_r experts, no bias)
+ * next to tile_counts[j, i] (required here).  "SMEBU Load Balancing" ("How it
+ * works") keeps a small sequence-wise balance loss, eqs. (29)-(32), with
+ * coefficient alpha; the pages do not print it, and it is read as the
+ * complementary sequence-wise balance loss of auxiliary-loss-free balancing
+ * (see seq_balance_loss).  The sums run in fp32 over the fp32 scores of the
+ * epilogue in a fixed order (deterministic); rows past T add nothing.
+ * tile_counts  device, int32 [ceil(T/128), N_r], written, not NULL.
+ * tile_psum    device, fp32 [ceil(T/128), N_r], written, not NULL.
+ * zloss_sum    device fp64 scalar (8-byte aligned, accumulated) or NULL.
+ * Other arguments and outputs as router_forward.
+ */
+int router_forward_balance(const uint16_t *hidden, const uint16_t *W_router, const float *bias,
+                           int T, int d, int N_r, int K,
+                           int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                           float *tile_psum, double *zloss_sum, int32_t *status, ebl_stream_t stream);
+
+/*
+ * seq_balance_loss -- the sequence-wise balance loss from the per-tile
+ * statistics of router_forward_balance.  For each sequence b of seq_len
+ * consecutive tokens (B = T / seq_len sequences, S = seq_len):
+ *   f_i = N_r / (K S) * (selections of expert i in the sequence)
+ *   P_i = (1 / S) * sum_t s_{t,i} / sum_l s_{t,l}
+ *   loss_seq[b] = alpha * sum_i f_i P_i           fp64
+ *   *loss = (1 / B) * sum_b loss_seq[b]           fp64, the batch value
+ * Passage: "SMEBU Load Balancing", "How it works" (the loss, eqs. (29)-(32),
+ * alpha = 5e-5 on the Large checkpoint); "Arcee Halts 400B Blackwell Model
+ * Collapse With Dynamic Router Biases", stabilization table (balancing
+ * evaluated per sequence).  The formula is a reading: the complementary
+ * sequence-wise balance loss published with auxiliary-loss-free balancing.
+ * Only the forward value is computed.
+ * tile_counts, tile_psum  device, [T/128, N_r] as router_forward_balance wrote them.
+ * T           tokens, a multiple of seq_len; T == 0 is a no-op.
+ * N_r, K      as for the router call that produced the statistics.
+ * seq_len     tokens per sequence, a positive multiple of 128.
+ * alpha       the coefficient (finite).
+ * loss_seq    device, fp64 [B], written (8-byte aligned).
+ * loss        device, fp64 scalar, written (8-byte aligned).
+ * Deterministic (fixed-order sums).  Two launches on `stream`.
+ */
+int seq_balance_loss(const int32_t *tile_counts, const float *tile_psum, int T, int N_r, int K, int seq_len,
+                     float alpha, double *loss_seq, double *loss, ebl_stream_t stream);
+
+/*
  * router_forward_logits -- the same selection, gates and counts from
  * precomputed fp32 logits.  This is the bit-exact mode: each value that
  * decides a selection has one defined rounding,

@@ -107,6 +107,26 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.ebl_check_finite_f32(ctypes.c_void_p(0x10002), 10, FAKE, None) == EINVAL   # not 4-byte aligned
     assert lib.ebl_check_finite_bf16(ctypes.c_void_p(0x10001), 10, FAKE, None) == EINVAL  # not 2-byte aligned
     assert lib.ebl_check_finite_bf16(None, 0, FAKE, None) == 0                              # empty: nothing to do
+    # sequence-wise balance: the option needs tile_counts and tile_psum; the loss
+    # wants seq_len a positive multiple of 128 that divides T
+    bal = lambda T=256, tc=FAKE, tp=FAKE: lib.router_forward_balance(FAKE, FAKE, FAKE, T, 256, 64, 4, FAKE, FAKE,
+                                                                     FAKE, tc, tp, None, None, None)
+    assert bal(tc=None) == EINVAL
+    assert bal(tp=None) == EINVAL
+    assert bal(tp=ctypes.c_void_p(0x10002)) == EINVAL
+    assert bal(T=0, tc=None, tp=None) == 0
+    sb = lambda T=1024, Nr=64, K=4, S=256, a=5e-5, ls=FAKE, l=FAKE: lib.seq_balance_loss(FAKE, FAKE, T, Nr, K, S, a,
+                                                                                         ls, l, None)
+    assert sb(S=100) == EINVAL
+    assert sb(S=0) == EINVAL
+    assert sb(T=1280, S=512) == EINVAL
+    assert sb(K=9) == EINVAL
+    assert sb(Nr=0) == EINVAL
+    assert sb(a=float("nan")) == EINVAL
+    assert sb(a=float("inf")) == EINVAL
+    assert sb(ls=None) == EINVAL
+    assert sb(l=ctypes.c_void_p(0x10004)) == EINVAL                                       # not 8-byte aligned
+    assert sb(T=0, ls=None, l=None) == 0                                                  # no tokens: nothing to do
 
 
 def test_binding_has_no_cpu_fallback():
