@@ -57,6 +57,46 @@ def test_router_full_size_sampled(cuda_device, name):
         assert int(counts[:8].sum().item()) == 0     # bias -1 keeps the 8 dead-start experts out
 
 
+def test_balance_option_full_tie_workload(cuda_device):
+    """The balance option on the 1M-token tie workload (the benchmark's
+    launch): routing bit-identical to router_forward; every tile's sums of
+    s / total equal its 128 tokens; sampled tiles and one whole 4096-token
+    sequence against the oracle (tolerances as in test_gpu_seq_balance)."""
+    from tests.test_gpu_seq_balance import PSUM_ATOL, PSUM_RTOL
+    cfg = synth.WORKLOADS["ties"]
+    T, d, Nr, K, S = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"], 4096
+    dev = cuda_device
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    h = synth.hidden_normal(T, d, seed=synth.step_seed("ties", 0), device=dev, quant8=True)
+    bias = synth.dead_start_bias(Nr, device=dev)
+    tiles = T // 128
+    c1 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    c2 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.empty(tiles, Nr, dtype=torch.int32, device=dev)
+    tp = torch.empty(tiles, Nr, device=dev)
+    idx, gates = ebl.router_forward_balance(h, W, bias, K, c1, tc, tp)
+    loss, loss_seq = ebl.seq_balance_loss(tc, tp, T, K, S, ebl.SEQ_BALANCE_ALPHA)
+    i2, g2 = ebl.router_forward(h, W, bias, K, c2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, i2) and torch.equal(gates, g2) and torch.equal(c1, c2)
+    assert float((tp.double().sum(1) - 128).abs().max()) < 128 * 1e-5
+    sample = sorted({0, tiles - 1} | set(np.random.default_rng(3).choice(tiles, 6, replace=False).tolist()))
+    rows = torch.cat([torch.arange(j * 128, (j + 1) * 128) for j in sample])
+    ref = oracle.router_gemm(h[rows.to(dev)].cpu(), W.cpu(), bias.cpu().numpy(), K, want_scores=True)
+    want = oracle.tile_psum(ref.scores, 128)
+    got = to_np(tp)[sample].astype(np.float64)
+    assert np.all(np.abs(got - want) <= PSUM_RTOL * want + PSUM_ATOL)
+    # the last sequence end to end
+    b = T // S - 1
+    hs = h[b * S:(b + 1) * S].cpu()
+    ref = oracle.router_gemm(hs, W.cpu(), bias.cpu().numpy(), K, want_scores=True)
+    r = oracle.seq_balance(ref.scores, ref.idx, S, ebl.SEQ_BALANCE_ALPHA)
+    excused = int((ref.gap < 1e-3).sum())
+    got = float(loss_seq[b].item())
+    assert abs(got - r.loss) <= 2e-5 * r.loss + excused * ebl.SEQ_BALANCE_ALPHA * Nr / S, (got, r.loss, excused)
+    assert abs(float(loss.item()) - float(loss_seq.mean().item())) <= 1e-15 * float(loss.item())
+
+
 def test_logits_mode_full_tie_workload(cuda_device):
     """The tie workload in logits mode at full size: bit-exact against the oracle."""
     cfg = synth.WORKLOADS["ties"]

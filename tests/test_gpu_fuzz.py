@@ -1,7 +1,8 @@
 """Seeded random shapes through every mode against the oracle (small sizes):
 logits mode bit-exact (both kernels: aligned and misaligned logits), GEMM mode
-under the near-tie rule, dispatch and combine bit-exact, and the bias updates
-(SMEBU clamped and linear over several layers, the sign update).  Each case
+under the near-tie rule, dispatch and combine bit-exact, the bias updates
+(SMEBU clamped and linear over several layers, the sign update), and the
+sequence-wise balance statistics.  Each case
 draws its sizes, the bias pattern and the value distribution from its own seed."""
 import numpy as np
 import pytest
@@ -161,3 +162,33 @@ def test_bias_updates_random(cuda_device, case):
     rc, mvo = oracle.sign_update(counts[-1], b, gamma)
     assert rel_err(to_np(b1), b).max() <= STATE_RTOL
     assert np.float32(mvo).tobytes() == to_np(mv1).tobytes()
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_balance_option_random_shapes(cuda_device, case):
+    """GEMM mode with the balance option on random shapes: tile_psum against
+    the oracle's per-tile sums, and the loss over random sequence lengths."""
+    from tests.test_gpu_seq_balance import PSUM_ATOL, PSUM_RTOL
+    rng = np.random.default_rng(9000 + case)
+    S = 128 * int(rng.integers(1, 5))
+    T = S * int(rng.integers(1, 6))
+    Nr = 32 * int(rng.integers(1, 9))
+    K = int(rng.integers(1, min(8, Nr) + 1))
+    d = 64 * int(rng.integers(1, 17))
+    dev = cuda_device
+    h = synth.hidden_normal(T, d, seed=9100 + case, quant8=bool(rng.integers(0, 2)))
+    W = synth.router_weight(Nr, d, seed=9200 + case)
+    b = _bias(rng, Nr)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.empty(T // 128, Nr, dtype=torch.int32, device=dev)
+    tp = torch.empty(T // 128, Nr, device=dev)
+    alpha = float(np.float32(10 ** rng.uniform(-5, -3)))
+    ebl.router_forward_balance(h.to(dev), W.to(dev), torch.from_numpy(b).to(dev), K, counts, tc, tp)
+    loss, loss_seq = ebl.seq_balance_loss(tc, tp, T, K, S, alpha)
+    torch.cuda.synchronize()
+    ref = oracle.router_gemm(h, W, b, K, want_scores=True)
+    want = oracle.tile_psum(ref.scores, 128)
+    assert np.all(np.abs(to_np(tp).astype(np.float64) - want) <= PSUM_RTOL * want + PSUM_ATOL)
+    r = oracle.seq_balance(ref.scores, ref.idx, S, alpha)
+    excused = (ref.gap < 1e-3).reshape(T // S, S).sum(1)
+    assert np.all(np.abs(to_np(loss_seq) - r.loss_seq) <= 2e-5 * r.loss_seq + excused * alpha * Nr / S)
