@@ -460,6 +460,15 @@ def main():
         extra["logits_mode"] = {"tokens_per_s": T * world / (lm / 1e3), "ms": lm,
                                 "achieved_gbs": lbytes / (lm / 1e3) / 1e9,
                                 "frac_hbm": lbytes / (lm / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        tpl = torch.empty((T + 127) // 128, Nr, dtype=torch.float32, device=dev)
+        ebl.balance_stats_logits(x, tile_psum=tpl, stream=stream)
+        ev[0].record(stream)
+        for _ in range(reps):
+            ebl.balance_stats_logits(x, tile_psum=tpl, stream=stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        extra["logits_mode"]["balance_stats_ms"] = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
+        del tpl
         counts.zero_()
         del x
 

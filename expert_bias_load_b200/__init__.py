@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_balance",
-    "seq_balance_loss", "router_forward_logits", "smebu_step",
+    "seq_balance_loss", "balance_stats_logits", "router_forward_logits", "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
     "read_internal_status", "check_finite", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD",
     "EBL_ST_TIMEOUT", "EBL_ST_BAD_COUNTS", "EBL_ST_NONFINITE",
@@ -57,6 +57,7 @@ SIGNATURES = {
     "router_forward_logits": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "router_forward_balance": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "seq_balance_loss": (_I, [_P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "balance_stats_logits": (_I, [_P, _I, _I, _P, _P]),
     "smebu_step": (_I, [_P, _P, _P, _I, _F, _F, _F, _I, _P, _P, _P]),
     "smebu_step_layers": (_I, [_P, _P, _P, _I, _I, _F, _F, _F, _I, _I, _P, _P, _P]),
     "sign_update_step": (_I, [_P, _P, _I, _F, _I, _P, _P, _P]),
@@ -218,6 +219,16 @@ def router_forward_balance(hidden, W_router, bias, K, counts, tile_counts, tile_
           _ptr(gates), _ptr(counts), _ptr(tile_counts), _ptr(tile_psum), _ptr(zloss_sum), _ptr(status),
           _stream(stream))
     return topk_idx, gates
+
+
+def balance_stats_logits(logits, tile_psum=None, stream=None):
+    """Logits mode: per-tile sums of s / sum_j s (s the fp64-rounded-once
+    score), fp32 [ceil(T/128), N_r].  Returns tile_psum."""
+    _check(logits, "logits", torch.float32)
+    T, Nr = logits.shape
+    tile_psum = _out(tile_psum, "tile_psum", ((T + 127) // 128, Nr), torch.float32, logits.device)
+    _call("balance_stats_logits", _ptr(logits), T, Nr, _ptr(tile_psum), _stream(stream))
+    return tile_psum
 
 
 def seq_balance_loss(tile_counts, tile_psum, T, K, seq_len, alpha=SEQ_BALANCE_ALPHA, loss_seq=None, loss=None,

@@ -193,6 +193,19 @@ int router_forward_balance(const uint16_t *hidden, const uint16_t *W_router, con
                             tile_psum, status, stream);
 }
 
+int balance_stats_logits(const float *logits, int T, int N_r, float *tile_psum, ebl_stream_t stream) {
+    if (check_T(T) || N_r < 1 || N_r > EBL_MAX_EXPERTS) return EBL_EINVAL;
+    if (T > 0 && (!logits || !tile_psum)) return EBL_EINVAL;
+    if (!aligned4(logits) || !aligned4(tile_psum)) return EBL_EINVAL;
+    if (T == 0) return EBL_OK;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    cudaError_t e = ebl::launch_tile_psum_logits(logits, T, N_r, tile_psum, di.num_sms,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
+}
+
 int seq_balance_loss(const int32_t *tile_counts, const float *tile_psum, int T, int N_r, int K, int seq_len,
                      float alpha, double *loss_seq, double *loss, ebl_stream_t stream) {
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;

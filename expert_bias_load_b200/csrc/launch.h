@@ -37,6 +37,10 @@ cudaError_t launch_smebu(int32_t *counts, float *bias, float *momentum, int L, i
 cudaError_t launch_sign_update(int32_t *counts, float *bias, int Nr, float gamma, int reset_counts,
                                float *maxvio_out, int32_t *status, cudaStream_t stream);
 
+// balance_logits.cu
+cudaError_t launch_tile_psum_logits(const float *logits, int T, int Nr, float *tile_psum, int num_sms,
+                                    cudaStream_t stream);
+
 // seq_balance.cu
 cudaError_t launch_seq_balance(const int32_t *tile_counts, const float *tile_psum, int T, int Nr, int K, int seq_len,
                                float alpha, double *loss_seq, double *loss, cudaStream_t stream);

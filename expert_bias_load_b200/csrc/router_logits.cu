@@ -31,18 +31,13 @@
 
 #include "launch.h"
 #include "ptx.cuh"
+#include "scores.cuh"
 #include "topk.cuh"
 
 namespace ebl {
 namespace {
 
 constexpr int kThreads = kTileTokens;  // one thread per row of a tile
-
-__device__ __forceinline__ float sigmoid_rounded_once(float x) {
-    // fp64 evaluation, one rounding to fp32 at the end
-    const double e = exp(-(double)x);
-    return __double2float_rn(__drcp_rn(__dadd_rn(1.0, e)));  // correctly rounded 1/y, the same as 1.0/y
-}
 
 // fp32 sigmoid from the fast intrinsics: __expf (at most 2 + 1.173|x| ulp off)
 // and __fdividef (at most 2 ulp).  Its distance to sigmoid_rounded_once() is

@@ -160,8 +160,27 @@ int router_forward_balance(const uint16_t *hidden, const uint16_t *W_router, con
                            float *tile_psum, double *zloss_sum, int32_t *status, ebl_stream_t stream);
 
 /*
+ * balance_stats_logits -- the per-tile statistics of the sequence-wise balance
+ * loss in logits mode (a separate pass over the logits):
+ *   tile_psum[j, i] = sum over tokens t in [128 j, 128 j + 128), t < T, of
+ *                     s_{t,i} / sum_l s_{t,l}
+ * with s = (float)(1 / (1 + exp(-(double)x))), the logits-mode score of
+ * router_forward_logits.  Row totals and the sums run in fp64 in a fixed
+ * order and are rounded once to fp32, so each output is within one fp32
+ * rounding of the exact value.  Pair it with the tile_counts of
+ * router_forward_logits and call seq_balance_loss.  Passage as for
+ * router_forward_balance.
+ * logits     device, fp32 [T, N_r], 4-byte aligned (assumed finite).
+ * T          tokens, 0 <= T <= 2^31 - 2^8; T == 0 is a no-op.
+ * N_r        1 <= N_r <= 256.
+ * tile_psum  device, fp32 [ceil(T/128), N_r], written.
+ */
+int balance_stats_logits(const float *logits, int T, int N_r, float *tile_psum, ebl_stream_t stream);
+
+/*
  * seq_balance_loss -- the sequence-wise balance loss from the per-tile
- * statistics of router_forward_balance.  For each sequence b of seq_len
+ * statistics of router_forward_balance (GEMM mode) or of
+ * router_forward_logits and balance_stats_logits (logits mode).  For each sequence b of seq_len
  * consecutive tokens (B = T / seq_len sequences, S = seq_len):
  *   f_i = N_r / (K S) * (selections of expert i in the sequence)
  *   P_i = (1 / S) * sum_t s_{t,i} / sum_l s_{t,l}

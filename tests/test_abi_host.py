@@ -127,6 +127,12 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert sb(ls=None) == EINVAL
     assert sb(l=ctypes.c_void_p(0x10004)) == EINVAL                                       # not 8-byte aligned
     assert sb(T=0, ls=None, l=None) == 0                                                  # no tokens: nothing to do
+    assert lib.balance_stats_logits(FAKE, 100, 0, FAKE, None) == EINVAL
+    assert lib.balance_stats_logits(FAKE, 100, 257, FAKE, None) == EINVAL
+    assert lib.balance_stats_logits(None, 100, 8, FAKE, None) == EINVAL
+    assert lib.balance_stats_logits(FAKE, 100, 8, None, None) == EINVAL
+    assert lib.balance_stats_logits(ctypes.c_void_p(0x10002), 100, 8, FAKE, None) == EINVAL
+    assert lib.balance_stats_logits(None, 0, 8, None, None) == 0
 
 
 def test_binding_has_no_cpu_fallback():

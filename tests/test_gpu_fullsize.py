@@ -98,7 +98,8 @@ def test_balance_option_full_tie_workload(cuda_device):
 
 
 def test_logits_mode_full_tie_workload(cuda_device):
-    """The tie workload in logits mode at full size: bit-exact against the oracle."""
+    """The tie workload in logits mode at full size: bit-exact against the
+    oracle, and the sequence-wise balance loss within one fp32 rounding."""
     cfg = synth.WORKLOADS["ties"]
     T, Nr, K = cfg["T"], cfg["Nr"], cfg["K"]
     dev = cuda_device
@@ -107,12 +108,22 @@ def test_logits_mode_full_tie_workload(cuda_device):
     counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
     tiles = torch.empty(((T + 127) // 128, Nr), dtype=torch.int32, device=dev)
     idx, gates = ebl.router_forward_logits(x, bias, K, counts, tile_counts=tiles)
+    tp = ebl.balance_stats_logits(x)
+    S = 4096
+    loss, loss_seq = ebl.seq_balance_loss(tiles, tp, T, K, S, ebl.SEQ_BALANCE_ALPHA)
     torch.cuda.synchronize()
-    ref = oracle.router_logits(to_np(x), to_np(bias), K, tile_tokens=128)
+    ref = oracle.router_logits(to_np(x), to_np(bias), K, tile_tokens=128, want_scores=True)
     assert np.array_equal(to_np(idx), ref.idx)
     assert np.array_equal(to_np(gates), ref.gates)
     assert np.array_equal(to_np(counts), ref.counts)
     assert np.array_equal(to_np(tiles), ref.tile_counts)
+    # the sequence-wise balance loss over 256 sequences of 4096 tokens (tolerances
+    # as in test_gpu_seq_balance: one fp32 rounding per tile sum)
+    scores = ref.scores.astype(np.float64)
+    want = oracle.tile_psum(scores, 128)
+    assert np.all(np.abs(to_np(tp).astype(np.float64) - want) <= 2.0 ** -23 * want)
+    r = oracle.seq_balance(scores, ref.idx, S, ebl.SEQ_BALANCE_ALPHA)
+    assert np.allclose(to_np(loss_seq), r.loss_seq, rtol=1.2e-7, atol=0)
 
 
 def test_dispatch_combine_full_size(cuda_device):

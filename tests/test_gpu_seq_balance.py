@@ -14,6 +14,11 @@ into the per-sequence and batch values.  Tolerances:
     tokens the near-tie rule excuses: moving one selection of a sequence from
     expert i to j changes its loss by alpha N_r / (K S^2) (q_j - q_i), at most
     alpha N_r / (K S) per moved selection.
+  - Logits mode: the scores have one defined rounding and the selections are
+    bit-exact, and balance_stats_logits sums in fp64 and rounds once, so each
+    tile_psum entry is within one fp32 rounding (2^-24 relative, taken as
+    2^-23 for the fp64 summation order) of the oracle, and the loss, a sum of
+    positive terms each off by at most that much, within 1.2e-7 relative.
 """
 import numpy as np
 import pytest
@@ -158,3 +163,44 @@ def test_empty_batch_is_a_noop(cuda_device):
     loss, loss_seq = ebl.seq_balance_loss(tc, tp, 0, 4, 128)
     torch.cuda.synchronize()
     assert idx.numel() == 0 and loss_seq.numel() == 0 and int(counts.sum().item()) == 0
+
+
+LOGITS_CASES = [(1000, 256, 4), (300, 7, 3), (129, 1, 1), (4096, 64, 8), (2000, 255, 2), (256, 33, 5)]
+
+
+@pytest.mark.parametrize("T,Nr,K", LOGITS_CASES)
+def test_logits_mode_tile_psum(cuda_device, T, Nr, K):
+    rng = np.random.default_rng(T + Nr)
+    x = (rng.standard_normal((T, Nr)) * 3).astype(np.float32)
+    x[: T // 3] = np.round(x[: T // 3] * 8) / 8                          # ties and repeated values
+    xd = torch.from_numpy(x).to(cuda_device)
+    tp = ebl.balance_stats_logits(xd)
+    torch.cuda.synchronize()
+    ref = oracle.router_logits(x, np.zeros(Nr, np.float32), K, want_scores=True)
+    want = oracle.tile_psum(ref.scores.astype(np.float64), 128)
+    got = to_np(tp).astype(np.float64)
+    err = np.abs(got - want)
+    assert np.all(err <= 2.0 ** -23 * want), (err / want).max()
+    print("logits-mode tile_psum max rel err %.3e (2^-24 = %.3e)" % ((err / want).max(), 2.0 ** -24))
+
+
+@pytest.mark.parametrize("T,Nr,K,S", [(4096, 256, 4, 1024), (1536, 64, 8, 512), (1280, 13, 2, 128)])
+def test_logits_mode_loss_end_to_end(cuda_device, T, Nr, K, S):
+    """Logits mode: exact selections and loads, so the loss has no excused tokens."""
+    rng = np.random.default_rng(3 * T + Nr)
+    x = np.round(rng.standard_normal((T, Nr)).astype(np.float32) * 8) / 8
+    b = (rng.integers(-2, 3, Nr) * 0.01).astype(np.float32)
+    dev = cuda_device
+    xd = torch.from_numpy(x).to(dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.empty(T // 128, Nr, dtype=torch.int32, device=dev)
+    ebl.router_forward_logits(xd, torch.from_numpy(b).to(dev), K, counts, tile_counts=tc)
+    tp = ebl.balance_stats_logits(xd)
+    alpha = ebl.SEQ_BALANCE_ALPHA
+    loss, loss_seq = ebl.seq_balance_loss(tc, tp, T, K, S, alpha)
+    torch.cuda.synchronize()
+    ref = oracle.router_logits(x, b, K, want_scores=True, tile_tokens=128)
+    assert np.array_equal(to_np(tc), ref.tile_counts)
+    r = oracle.seq_balance(ref.scores.astype(np.float64), ref.idx, S, alpha)
+    assert np.allclose(to_np(loss_seq), r.loss_seq, rtol=1.2e-7, atol=0), (to_np(loss_seq), r.loss_seq)
+    assert abs(float(loss.item()) - r.loss) <= 1.2e-7 * r.loss
