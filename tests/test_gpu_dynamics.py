@@ -130,6 +130,60 @@ def test_router_step_in_cuda_graph(cuda_device):
         assert torch.equal(a, c)
 
 
+def test_balance_step_in_cuda_graph(cuda_device):
+    """The training-side router step with both auxiliary statistics -- router
+    with the z-loss and balance options, the sequence-wise balance loss, SMEBU
+    -- captured once in a CUDA graph: replays leave the same bias, momentum,
+    indices and per-tile sums, and the same loss values, as eager launches
+    (the z-loss sum up to the order of its fp64 atomics)."""
+    dev = cuda_device
+    T, d, Nr, K, S = 4096, 512, 256, 4, 1024
+    W = synth.router_weight(Nr, d, seed=31).to(dev)
+    h = synth.hidden_normal(T, d, seed=32, device=dev)
+    state = {}
+    for mode in ("eager", "graph"):
+        b = synth.dead_start_bias(Nr, device=dev)
+        m = torch.zeros(Nr, device=dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        g = torch.empty(T, K, device=dev)
+        tc = torch.empty(T // 128, Nr, dtype=torch.int32, device=dev)
+        tp = torch.empty(T // 128, Nr, device=dev)
+        z = torch.zeros(1, dtype=torch.float64, device=dev)
+        lseq = torch.empty(T // S, dtype=torch.float64, device=dev)
+        loss = torch.empty(1, dtype=torch.float64, device=dev)
+
+        def step(stream=None):
+            z.zero_()
+            ebl.router_forward_balance(h, W, b, K, counts, tc, tp, zloss_sum=z, topk_idx=idx, gates=g,
+                                       stream=stream)
+            ebl.seq_balance_loss(tc, tp, T, K, S, loss_seq=lseq, loss=loss, stream=stream)
+            ebl.smebu_step(counts, b, m, reset_counts=True, stream=stream)
+
+        if mode == "eager":
+            for _ in range(4):
+                step()
+        else:
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                step(s)                               # warm-up launch outside the graph
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(torch.cuda.current_stream())
+            for _ in range(3):
+                graph.replay()
+        torch.cuda.synchronize()
+        state[mode] = (b.clone(), m.clone(), idx.clone(), g.clone(), tp.clone(), lseq.clone(), loss.clone(),
+                       float(z.item()))
+    for a, c in zip(state["eager"][:-1], state["graph"][:-1]):
+        assert torch.equal(a, c)
+    ze, zg = state["eager"][-1], state["graph"][-1]
+    assert abs(ze - zg) <= 1e-12 * ze
+
+
 def test_full_step_in_cuda_graph(cuda_device):
     """Router with tile counts, SMEBU, dispatch and combine captured once in a
     CUDA graph: replays give the same bias, indices, dispatched rows and
