@@ -12,7 +12,8 @@ public binding, so it is also the command to put under a profiler: with
 Entry points: router (GEMM mode), zloss (GEMM mode with the z-loss), balance
 (GEMM mode with the sequence-wise balance statistics, then the loss over
 sequences of 4096 tokens, or of T tokens when T is smaller), logits (logits
-mode), smebu, sign, dispatch, combine.  For the one-CTA update kernels
+mode), balance_logits (the logits-mode balance statistics), smebu, sign,
+dispatch, combine.  For the one-CTA update kernels
 (smebu, sign) the time per call is the host's launch rate, not the kernel's.
 """
 from __future__ import annotations
@@ -40,7 +41,8 @@ def _time(fn, warmup, reps):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("op", choices=["router", "zloss", "balance", "logits", "smebu", "sign", "dispatch", "combine"])
+    ap.add_argument("op", choices=["router", "zloss", "balance", "logits", "balance_logits", "smebu", "sign", "dispatch",
+                                   "combine"])
     ap.add_argument("--tokens", type=int, default=1 << 20)
     ap.add_argument("--hidden", type=int, default=4096)
     ap.add_argument("--experts", type=int, default=256)
@@ -86,6 +88,12 @@ def main(argv=None):
         fn = lambda: ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=g)
         ms = _time(fn, a.warmup, a.reps)
         work = "%.1f GB/s" % ((T * Nr * 4 + T * K * 8) / ms / 1e6)
+    elif a.op == "balance_logits":
+        x = synth.logits_normal(T, Nr, seed=a.seed, device=dev, quant8=True)
+        tp = torch.empty((T + 127) // 128, Nr, device=dev)
+        fn = lambda: ebl.balance_stats_logits(x, tile_psum=tp)
+        ms = _time(fn, a.warmup, a.reps)
+        work = "%.1f G scores/s" % (T * Nr / ms / 1e6)
     elif a.op in ("smebu", "sign"):
         counts.copy_(torch.randint(0, 2 * T * K // Nr + 1, (Nr,), generator=torch.Generator().manual_seed(a.seed),
                                    dtype=torch.int32).to(dev))

@@ -283,8 +283,8 @@ def test_logits_mode_saturated_scores(cuda_device, misalign):
 
 def test_microbench_runs_every_entry_point(cuda_device, capsys):
     from expert_bias_load_b200 import microbench
-    for op in ("router", "zloss", "balance", "logits", "smebu", "sign", "dispatch", "combine"):
+    for op in ("router", "zloss", "balance", "logits", "balance_logits", "smebu", "sign", "dispatch", "combine"):
         microbench.main([op, "--tokens", "4096", "--hidden", "256", "--experts", "64", "--topk", "4",
                          "--warmup", "1", "--reps", "2"])
     lines = [l for l in capsys.readouterr().out.splitlines() if " ms, " in l]
-    assert len(lines) == 8
+    assert len(lines) == 9

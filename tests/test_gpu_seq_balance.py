@@ -173,6 +173,7 @@ def test_logits_mode_tile_psum(cuda_device, T, Nr, K):
     rng = np.random.default_rng(T + Nr)
     x = (rng.standard_normal((T, Nr)) * 3).astype(np.float32)
     x[: T // 3] = np.round(x[: T // 3] * 8) / 8                          # ties and repeated values
+    x[T // 2, : min(Nr, 6)] = [88.7, -88.7, -103.0, -104.0, 700.0, -3e38][: min(Nr, 6)]   # saturated, subnormal
     xd = torch.from_numpy(x).to(cuda_device)
     tp = ebl.balance_stats_logits(xd)
     torch.cuda.synchronize()
