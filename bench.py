@@ -156,8 +156,12 @@ class OracleSample:
         return time.perf_counter() - t0
 
     def rows_for(self, seconds):
+        # a 64-row probe overstates the time per row (thread start-up), so a
+        # second probe of about a tenth of the target refines the estimate
         t = self.run(64, seed=1)
-        return int(max(16, min(self.cfg["T"], 64 * seconds / max(t, 1e-4))))
+        rows = int(max(64, min(self.cfg["T"], 64 * seconds / 10 / max(t, 1e-4))))
+        t = self.run(rows, seed=2)
+        return int(max(16, min(self.cfg["T"], rows * seconds / max(t, 1e-4))))
 
 
 def oracle_sample(cfg, seconds, seed=0):
