@@ -162,7 +162,7 @@ __device__ __forceinline__ void column_fold(float (&v)[kChunk], int lane) {
 }
 
 // Sums over the warp's 32 rows of the 16 columns in v (this lane's row):
-// lanes 2c and 2c + 1 return the sum of column c.  31 shuffles per 16 columns.
+// lanes 2c and 2c + 1 return the sum of column c.  16 shuffles per 16 columns.
 __device__ __forceinline__ float warp_column_sums(float (&v)[kChunk], int lane) {
     column_fold<8>(v, lane);
     column_fold<4>(v, lane);
