@@ -141,3 +141,13 @@ def test_binding_has_no_cpu_fallback():
     with pytest.raises(ValueError):
         ebl.router_forward(h, torch.zeros(32, 64, dtype=torch.bfloat16), torch.zeros(32), 2,
                            torch.zeros(32, dtype=torch.int32))
+    # the balance entry points refuse host tensors too
+    tc = torch.zeros(1, 32, dtype=torch.int32)
+    tp = torch.zeros(1, 32)
+    with pytest.raises(ValueError):
+        ebl.router_forward_balance(h, torch.zeros(32, 64, dtype=torch.bfloat16), torch.zeros(32), 2,
+                                   torch.zeros(32, dtype=torch.int32), tc, tp)
+    with pytest.raises(ValueError):
+        ebl.balance_stats_logits(torch.zeros(4, 32))
+    with pytest.raises(ValueError):
+        ebl.seq_balance_loss(tc, tp, 128, 2, 128)
