@@ -11,10 +11,13 @@
  *   "SMEBU Load Balancing" (study note), "How it works": eq. (17) bias only
  *     inside Top-K; eqs. (20)-(22) sign update with re-centred bias;
  *     eqs. (23)-(28) normalised violation, tanh clamp, scaled and re-centred
- *     step, momentum, bias add.
+ *     step, momentum, bias add; the sequence-wise balance loss, eqs.
+ *     (29)-(32), with alpha = 5e-5 (named, not printed: see
+ *     router_forward_balance for the reading).
  *   "Arcee Halts 400B Blackwell Model Collapse With Dynamic Router Biases",
  *     "The MaxVio Metric and the Day-4 Crisis": MaxVio, the ratio of the most-
- *     to the least-routed expert's load.
+ *     to the least-routed expert's load; the stabilization table: the z-loss
+ *     log^2 sum_i e^{x_i} and an auxiliary balance loss evaluated per sequence.
  *
  * Conventions shared by every entry point:
  *   - Pointers marked "device" are CUDA device pointers (or managed memory) on
