@@ -16,8 +16,9 @@
  *     router_forward_balance for the reading).
  *   "Arcee Halts 400B Blackwell Model Collapse With Dynamic Router Biases",
  *     "The MaxVio Metric and the Day-4 Crisis": MaxVio, the ratio of the most-
- *     to the least-routed expert's load; the stabilization table: the z-loss
- *     log^2 sum_i e^{x_i} and an auxiliary balance loss evaluated per sequence.
+ *     to the least-routed expert's load; and the stabilization table of
+ *     "Precision Fallbacks, Loss Stabilization, and MaxVio as Data Telemetry":
+ *     the z-loss log^2 sum_i e^{x_i}, an auxiliary balance loss per sequence.
  *
  * Conventions shared by every entry point:
  *   - Pointers marked "device" are CUDA device pointers (or managed memory) on
