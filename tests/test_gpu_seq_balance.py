@@ -6,7 +6,7 @@ into the per-sequence and batch values.  Tolerances:
   - tile_psum: the epilogue's scores are fp32 sigmoids (fast exp and
     reciprocal, a few ulp) of fp32-accumulated logits; s / total and the
     fixed-order fp32 sums over 128 rows add a few ulp more.  Each entry is
-    within 2e-5 relative (+1e-6 absolute per tile) of the fp64 oracle; the
+    within 2e-5 relative (+1e-6 absolute per token of the tile) of the fp64 oracle; the
     measured error is printed.
   - seq_balance_loss on given statistics: fp64 sums in another order than the
     oracle's, 1e-12 relative.
