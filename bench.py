@@ -39,6 +39,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-full-step", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--suite-seconds", type=float, default=3.0,
+                    help="target CPU time of each oracle sample of the per-workload suite (0: skip the suite)")
+    ap.add_argument("--suite-cpu-only", type=int, default=0, help=argparse.SUPPRESS)
     ap.add_argument("--tokens", type=int, default=0,
                     help="tokens per GPU (default: the tie workload's 1,048,576); smaller values are for profiling")
     return ap.parse_args()
@@ -173,10 +176,180 @@ def oracle_sample(cfg, seconds, seed=0):
     return rows / t, rows, o.threads, t
 
 
+# ------------------------------------------------ oracle on every workload
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# (workload, mode, timed on one thread, timed on all cores)
+SUITE_ENTRIES = [
+    ("tiny", "gemm", True, True), ("mid", "gemm", True, True), ("drift", "gemm", True, True),
+    ("dispatch", "gemm", False, True), ("ties", "logits", False, True), ("dispatch", "dispatch", False, True),
+]
+
+
+def suite_cpu(seconds, threads_label):
+    """CPU half of the suite, run in a child process whose OMP_NUM_THREADS
+    fixes the oracle's threads: per entry, the rows timed and the seconds.
+    Each sample is sized for about `seconds`; a sample smaller than the
+    workload is extrapolated linearly (tokens/s)."""
+    import numpy as np
+    import oracle
+    import synth
+    oracle.build()
+    out = []
+    for name, mode, one, allc in SUITE_ENTRIES:
+        if not (one if threads_label == "one_thread" else allc):
+            continue
+        c = synth.WORKLOADS[name]
+        T, d, Nr, K = c["T"], c["d"], c["Nr"], c["K"]
+        cap = T
+        if mode == "gemm":
+            W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d)
+
+            def run(rows, seed):
+                h = synth.hidden_normal(rows, d, seed=seed)
+                b = np.zeros(Nr, np.float32)
+                m = np.zeros(Nr, np.float32)
+                t0 = time.perf_counter()
+                r = oracle.router_gemm(h, W, b, K)
+                oracle.smebu(r.counts, b, m)
+                return time.perf_counter() - t0
+        elif mode == "logits":
+            def run(rows, seed):
+                x = synth.logits_normal(rows, Nr, seed=seed, quant8=True).numpy()
+                b = synth.dead_start_bias(Nr).numpy()
+                m = np.zeros(Nr, np.float32)
+                t0 = time.perf_counter()
+                r = oracle.router_logits(x, b, K)
+                oracle.smebu(r.counts, b, m)
+                return time.perf_counter() - t0
+        else:  # dispatch, identity expert, combine; host memory bounds the sample
+            cap = min(T, 16384)
+
+            def run(rows, seed):
+                h = synth.hidden_normal(rows, d, seed=seed)
+                r = oracle.router_logits(synth.logits_normal(rows, Nr, seed=seed + 1).numpy(),
+                                         np.zeros(Nr, np.float32), K)
+                t0 = time.perf_counter()
+                _, perm, dest = oracle.dispatch(r.idx, Nr)
+                X = oracle.gather_rows(h, perm)
+                oracle.combine(X, r.gates, dest, want64=False, want32=True)
+                return time.perf_counter() - t0
+        rows = min(64, cap)  # grow the sample until it takes a measurable share of the budget
+        t = run(rows, 1)
+        while t < seconds / 8 and rows < cap:
+            rows = min(cap, rows * max(2, int(seconds / 8 / max(t, 1e-6))))
+            t = run(rows, 1)
+        rows = int(min(cap, max(1, rows * seconds / max(t, 1e-6))))
+        t = run(rows, 2)
+        out.append({"workload": name, "mode": mode, "rows": rows, "seconds": t, "tokens_per_s": rows / t,
+                    "extrapolated": rows < T})
+    return out
+
+
+def cpu_baseline_suite(seconds, dev):
+    """The oracle on every workload (one thread on tiny, mid and drift; all
+    host cores on those, on the dispatch workload's router, on the tie
+    workload in logits mode and on dispatch + combine), each beside the GPU
+    path's tokens/s on the same configuration with inputs resident."""
+    import torch
+    import expert_bias_load_b200 as ebl
+    import synth
+    cpu = {}
+    for label, threads in (("one_thread", 1), ("all_cores", os.cpu_count() or 1)):
+        env = dict(os.environ, OMP_NUM_THREADS=str(threads))
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--suite-cpu-only",
+                            "1" if label == "one_thread" else "2", "--suite-seconds", str(seconds)],
+                           env=env, cwd=ROOT, capture_output=True, text=True, check=True)
+        cpu[label] = (threads, json.loads(r.stdout.strip().splitlines()[-1]))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def gpu_ms(fn, warmup=3, reps=10):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev[0].record()
+        for _ in range(reps):
+            fn()
+        ev[1].record()
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1]) / reps
+
+    entries = []
+    for name, mode, _, _ in SUITE_ENTRIES:
+        c = synth.WORKLOADS[name]
+        T, d, Nr, K = c["T"], c["d"], c["Nr"], c["K"]
+        bias = synth.dead_start_bias(Nr, device=dev) if name == "ties" else torch.zeros(Nr, device=dev)
+        m = torch.zeros(Nr, device=dev)
+        counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        g = torch.empty(T, K, device=dev)
+        if mode == "gemm":
+            h = synth.hidden_normal(T, d, seed=synth.step_seed(name, 0), device=dev)
+            W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+
+            def fn():
+                ebl.router_forward(h, W, bias, K, counts, topk_idx=idx, gates=g)
+                ebl.smebu_step(counts, bias, m, reset_counts=True)
+            what = "router (GEMM mode) + SMEBU"
+        elif mode == "logits":
+            x = synth.logits_normal(T, Nr, seed=synth.step_seed(name, 0), device=dev, quant8=True)
+
+            def fn():
+                ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=g)
+                ebl.smebu_step(counts, bias, m, reset_counts=True)
+            what = "router (logits mode) + SMEBU"
+        else:
+            h = synth.hidden_normal(T, d, seed=synth.step_seed(name, 0), device=dev)
+            x = synth.logits_normal(T, Nr, seed=synth.step_seed(name, 0) + 1, device=dev)
+            tiles = torch.empty((T + 127) // 128, Nr, dtype=torch.int32, device=dev)
+            ebl.router_forward_logits(x, torch.zeros(Nr, device=dev), K, counts, topk_idx=idx, gates=g,
+                                      tile_counts=tiles)
+            del x
+            offsets, perm, dest, X = ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles)
+            ws = torch.empty(max(16, ebl.dispatch_workspace_bytes(T, Nr)), dtype=torch.uint8, device=dev)
+            out = torch.empty(T, d, device=dev)
+
+            def fn():
+                ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles, offsets=offsets, perm=perm, dest=dest,
+                                 dispatched=X, workspace=ws)
+                ebl.moe_combine(X, g, dest, out=out)
+            what = "dispatch + identity expert + combine"
+        ms = gpu_ms(fn)
+        gpu_tps = T / (ms / 1e3)
+        e = {"workload": name, "T": T, "d": d, "N_r": Nr, "K": K, "step": what, "gpu_tokens_per_s": gpu_tps,
+             "gpu_ms": ms}
+        for label, (threads, res) in cpu.items():
+            for r in res:
+                if r["workload"] == name and r["mode"] == mode:
+                    e["oracle_" + label] = {"threads": threads, "rows": r["rows"], "seconds": r["seconds"],
+                                            "tokens_per_s": r["tokens_per_s"], "extrapolated": r["extrapolated"]}
+                    e["gpu_over_oracle_" + label] = gpu_tps / r["tokens_per_s"]
+        entries.append(e)
+        del fn
+        torch.cuda.empty_cache()
+    return {"entries": entries, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "note": "oracle samples sized for about %.0f s each; a sample smaller than T is extrapolated "
+                    "linearly; GPU inputs resident" % seconds}
+
+
 # ------------------------------------------------------------------- GPU leg
 
 def main():
     args = parse()
+    if args.suite_cpu_only:
+        print(json.dumps(suite_cpu(args.suite_seconds, "one_thread" if args.suite_cpu_only == 1 else "all_cores")),
+              flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -477,11 +650,16 @@ def main():
         del x
 
     cpu = None
+    suite = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, rows, threads, secs = oracle_sample(cfg, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": "%d rows of the tie workload (fp64 router GEMM + top-K + gates + counts, then SMEBU), "
-                         "%.1f s" % (rows, secs)}
+                         "%.1f s" % (rows, secs), "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+        if args.suite_seconds > 0 and args.tokens == 0:
+            del h
+            torch.cuda.empty_cache()
+            suite = cpu_baseline_suite(args.suite_seconds, dev)
 
     if world > 1:
         dist.barrier()
@@ -492,7 +670,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-            "clocks": clk, "status": st, "maxvio_after_warmup": maxvio_first, "full_step": full, **extra}
+            "clocks": clk, "status": st, "maxvio_after_warmup": maxvio_first, "full_step": full, **extra,
+            "cpu_baseline_suite": suite}
     print(json.dumps(line), flush=True)
 
 

@@ -223,7 +223,6 @@ int seq_balance_loss(const int32_t *tile_counts, const float *tile_psum, int T, 
 int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K, int32_t *topk_idx,
                           float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status,
                           ebl_stream_t stream) {
-    (void)status;  // no device-side error condition in this mode
     if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
     if (!bias || !counts) return EBL_EINVAL;
     if (T > 0 && (!logits || !topk_idx || !gates)) return EBL_EINVAL;  // T-sized buffers may be NULL when T == 0
@@ -235,7 +234,8 @@ int router_forward_logits(const float *logits, const float *bias, int T, int N_r
     int rc = device_info(&di);
     if (rc) return rc;
     cudaError_t e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts,
-                                              di.num_sms, reinterpret_cast<cudaStream_t>(stream));
+                                              status ? status : di.internal_status, di.num_sms,
+                                              reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 

@@ -271,9 +271,11 @@ __global__ void __launch_bounds__(32) copy_kernel(const uint8_t *__restrict__ hi
     if (lane == 0) {
         if (u < U) {
             // a load never landed: report, then give the loads already issued a
-            // bounded time to land before the shared memory goes away
+            // bounded time to land before the shared memory goes away.  The
+            // iteration that gave up had issued chunk u + kCopyAhead before its
+            // wait, so chunks u .. u + kCopyAhead (those below U) are in flight.
             atomicOr(status, kStTimeout);
-            const int64_t issued = min(U, u + kCopyAhead);
+            const int64_t issued = min(U, u + kCopyAhead + 1);
             for (int64_t w = u; w < issued; ++w)
                 mbar_wait(&full[w % kCopyStages], (uint32_t)((w / kCopyStages) & 1), &abort_flag, 100000000ull);
         }

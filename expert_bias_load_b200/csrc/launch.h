@@ -23,7 +23,7 @@ cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tma
 
 // router_logits.cu
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
-                                 float *gates, int32_t *counts, int32_t *tile_counts, int num_sms,
+                                 float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms,
                                  cudaStream_t stream);
 cudaError_t launch_score_error(const float *x, int64_t n, float *max_err, float *exact_out, cudaStream_t stream);
 cudaError_t launch_check_finite(const void *p, int64_t n, int bf16, int32_t *status, int num_sms,

@@ -15,6 +15,7 @@ constexpr int kStBadDest = 2;
 constexpr int kStEmptyLoad = 4;
 constexpr int kStTimeout = 8;
 constexpr int kStBadCounts = 16;
+constexpr int kStNonfinite = 32;
 
 // Upper bound on any single pipeline wait inside a kernel.  Correct runs wait
 // microseconds; after this the waiting role reports EBL_ST_TIMEOUT and bails.

@@ -530,9 +530,15 @@ __global__ void __launch_bounds__(threads_of(G), 1)
                         og[k] = tk.score[k] * inv;
                     }
                 }
+                bool unfilled = false;
 #pragma unroll
-                for (int k = 0; k < K; ++k)  // a non-finite row can leave a slot unfilled
-                    if ((unsigned)tk.idx[k] < (unsigned)Nr) atomicAdd(&hist[tk.idx[k]], 1);
+                for (int k = 0; k < K; ++k) {  // only a NaN or -inf key can leave a slot unfilled
+                    if ((unsigned)tk.idx[k] < (unsigned)Nr)
+                        atomicAdd(&hist[tk.idx[k]], 1);
+                    else
+                        unfilled = true;
+                }
+                if (unfilled) atomicOr(status, kStNonfinite);
             }
             if (want_tiles) {
                 mbar_arrive(epi_sync);

@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
                                                                  int32_t *__restrict__ topk_idx,
                                                                  float *__restrict__ gates,
                                                                  int32_t *__restrict__ counts,
-                                                                 int32_t *__restrict__ tile_counts) {
+                                                                 int32_t *__restrict__ tile_counts,
+                                                                 int32_t *__restrict__ status) {
     __shared__ float bias_s[kMaxExperts];
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
@@ -186,7 +187,10 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
                 for (int k = 0; k < K; ++k) {
                     oi[k] = tk.idx[k];
                     og[k] = __double2float_rn(__ddiv_rn((double)tk.score[k], sum));
-                    if ((unsigned)tk.idx[k] < (unsigned)Nr) atomicAdd(&hist[tk.idx[k]], 1);
+                    if ((unsigned)tk.idx[k] < (unsigned)Nr)
+                        atomicAdd(&hist[tk.idx[k]], 1);
+                    else
+                        atomicOr(status, kStNonfinite);  // only a NaN or -inf key leaves a slot unfilled
                 }
             }
         }
@@ -274,7 +278,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                                                                      int32_t *__restrict__ topk_idx,
                                                                      float *__restrict__ gates,
                                                                      int32_t *__restrict__ counts,
-                                                                     int32_t *__restrict__ tile_counts) {
+                                                                     int32_t *__restrict__ tile_counts,
+                                                                     int32_t *__restrict__ status) {
     // lane-local lists of the approximate pass hold P >= K values (P a power of two)
     constexpr int P = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
     constexpr int kRow = 32 * NV;  // floats per row in the ring (N_r rounded up, zero-filled)
@@ -539,15 +544,24 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
             }
         }
 
-        // gates (fp64, slot order), outputs, histogram: lane j writes slot j
+        // gates (fp64, slot order), outputs, histogram: lane j writes slot j.
+        // Slots [0, min(K, row_n)) hold the row's Top-K; fewer than K
+        // candidates happen only when NaN or -inf keys leave slots unfilled.
         if (row < T && j < K) {
             double sum = 0.0;
 #pragma unroll
-            for (int k = 0; k < K; ++k) sum = __dadd_rn(sum, (double)ss[k]);
-            const int c = sc[j];
-            topk_idx[row * K + j] = c;
-            gates[row * K + j] = __double2float_rn(__ddiv_rn((double)ss[j], sum));
-            if ((unsigned)c < (unsigned)Nr) atomicAdd(&hist[c], 1);
+            for (int k = 0; k < K; ++k)
+                if (k < row_n) sum = __dadd_rn(sum, (double)ss[k]);
+            if (j < row_n) {
+                const int c = sc[j];
+                topk_idx[row * K + j] = c;
+                gates[row * K + j] = __double2float_rn(__ddiv_rn((double)ss[j], sum));
+                atomicAdd(&hist[c], 1);
+            } else {
+                topk_idx[row * K + j] = 0x7fffffff;
+                gates[row * K + j] = 0.0f;
+                atomicOr(status, kStNonfinite);
+            }
         }
         __syncwarp();  // the ring stage and the candidate slots are reused
 
@@ -620,7 +634,7 @@ cudaError_t vec_setup(const void *kern, size_t smem, int *blocks_per_sm) {
 
 template <int K, int NV, bool FULL>
 cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, int32_t *topk_idx, float *gates,
-                       int32_t *counts, int32_t *tile_counts, int num_sms, cudaStream_t stream) {
+                       int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms, cudaStream_t stream) {
     const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL>);
     const size_t smem = vec_ring_bytes<NV>();
     int per_sm = 1;
@@ -630,14 +644,14 @@ cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, in
     int grid = num_sms * per_sm;
     if (grid > num_tiles) grid = num_tiles;
     router_logits_vec_kernel<K, NV, FULL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates,
-                                                                            counts, tile_counts);
+                                                                            counts, tile_counts, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
-                                 float *gates, int32_t *counts, int32_t *tile_counts, int num_sms,
+                                 float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms,
                                  cudaStream_t stream) {
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     if (Nr % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
@@ -647,8 +661,8 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
 #define EBL_VCASE(KK, NN) \
     case KK * 16 + NN:    \
         return Nr == 32 * NN                                                                                   \
-                   ? launch_vec<KK, NN, true>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream) \
-                   : launch_vec<KK, NN, false>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, num_sms, stream);
+                   ? launch_vec<KK, NN, true>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, status, num_sms, stream) \
+                   : launch_vec<KK, NN, false>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, status, num_sms, stream);
 #define EBL_VCASES(KK) EBL_VCASE(KK, 2) EBL_VCASE(KK, 4) EBL_VCASE(KK, 8)
             EBL_VCASES(1)
             EBL_VCASES(2)
@@ -671,7 +685,7 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
 #define EBL_CASE(KK)                                                                                    \
     case KK:                                                                                            \
         router_logits_kernel<KK><<<grid, kThreads, 0, stream>>>(logits, bias, T, Nr, topk_idx, gates, \
-                                                                counts, tile_counts);                  \
+                                                                counts, tile_counts, status);          \
         break;
         EBL_CASE(1)
         EBL_CASE(2)

@@ -53,12 +53,29 @@ class DataParallelRouterStep:
 
 
 def cuda_step(W_router, K, lam=5e-4, beta=0.5, kappa=2.0, group=None, stream=None):
-    """The step on the CUDA library: router_forward (GEMM mode), an all-reduce
-    of the loads, smebu_step with reset_counts so the next step starts at 0."""
+    """The step on the CUDA library: router_forward (GEMM mode) on this rank's
+    hidden states, an all-reduce of the loads, smebu_step with reset_counts so
+    the next step starts at 0."""
     import expert_bias_load_b200 as ebl
 
     def route(hidden, bias, counts):
         return ebl.router_forward(hidden, W_router, bias, K, counts, stream=stream)
+
+    def update(counts, bias, momentum, maxvio):
+        ebl.smebu_step(counts, bias, momentum, lam, beta, kappa, reset_counts=True, maxvio=maxvio, stream=stream)
+
+    return DataParallelRouterStep(route, update, group, stream)
+
+
+def cuda_logits_step(K, lam=5e-4, beta=0.5, kappa=2.0, group=None, stream=None):
+    """The same step fed with this rank's precomputed fp32 router logits
+    (router_forward_logits, the bit-exact mode): the global loads, and with
+    them bias and momentum, equal those of one process that routes the
+    concatenated batch."""
+    import expert_bias_load_b200 as ebl
+
+    def route(logits, bias, counts):
+        return ebl.router_forward_logits(logits, bias, K, counts, stream=stream)
 
     def update(counts, bias, momentum, maxvio):
         ebl.smebu_step(counts, bias, momentum, lam, beta, kappa, reset_counts=True, maxvio=maxvio, stream=stream)

@@ -65,7 +65,8 @@ typedef struct CUstream_st *ebl_stream_t;
 #define EBL_ST_EMPTY_LOAD 4   /* sum of loads was 0: bias/momentum left untouched */
 #define EBL_ST_TIMEOUT 8      /* a pipeline wait (router kernel, dispatch copy) ran out; outputs invalid */
 #define EBL_ST_BAD_COUNTS 16  /* dispatch: tile_counts do not add up to T*K (they do not match topk_idx) */
-#define EBL_ST_NONFINITE 32   /* ebl_check_finite_*: a NaN or infinity was found */
+#define EBL_ST_NONFINITE 32   /* ebl_check_finite_*: a NaN or infinity was found; routers: a Top-K slot
+                                 stayed unfilled (only a NaN or -inf key can cause that) */
 
 #define EBL_MAX_EXPERTS 256   /* N_r limit of every entry point */
 #define EBL_MAX_TOPK 8        /* K limit */
@@ -113,7 +114,10 @@ int ebl_tile_tokens(void);
  * counts       device, int32 [N_r], accumulated with one atomic per expert per CTA.
  * tile_counts  device, int32 [ceil(T/128), N_r], written; or NULL to skip.
  * status       device int32 or NULL; EBL_ST_TIMEOUT if the pipeline stalled.
- * Inputs are assumed finite.  Deterministic: the outputs do not depend on
+ * Inputs are assumed finite (ebl_check_finite_* can vouch for them).  If a
+ * NaN logit or a -inf bias leaves fewer than K experts with a key above -inf,
+ * the unfilled slots get expert id 0x7fffffff, add no load, and
+ * EBL_ST_NONFINITE is raised in status.  Deterministic: the outputs do not depend on
  * scheduling (integer histogram, per-row arithmetic in a fixed order).
  */
 int router_forward(const uint16_t *hidden, const uint16_t *W_router, const float *bias,
@@ -223,7 +227,9 @@ int seq_balance_loss(const int32_t *tile_counts, const float *tile_psum, int T, 
  *         16-byte aligned base the logits are read from HBM once; otherwise
  *         a slower kernel reads them twice (same results).
  * N_r     1 <= N_r <= 256 (any value).  K: 1 <= K <= min(8, N_r).
- * Other arguments as router_forward.  Logits and bias are assumed finite.
+ * Other arguments as router_forward.  Logits and bias are assumed finite;
+ * a Top-K slot that no key fills is reported as for router_forward
+ * (id 0x7fffffff, no load, EBL_ST_NONFINITE).
  */
 int router_forward_logits(const float *logits, const float *bias, int T, int N_r, int K,
                           int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,

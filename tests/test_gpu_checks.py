@@ -12,6 +12,8 @@ import torch
 
 import expert_bias_load_b200 as ebl
 import oracle
+import synth
+from tests.parity import to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -68,3 +70,61 @@ def test_exact_scores_match_the_oracle(cuda_device):
           % (mismatches, x.numel(), err, bound))
     assert mismatches == 0
     assert err * 4 <= bound
+
+
+@pytest.mark.parametrize("mode", ["gemm", "logits_vec", "logits_row"])
+def test_unfilled_slots_are_reported(cuda_device, mode):
+    """A bias of -inf on all but two experts leaves K = 4 slots with only two
+    keys above -inf: those two fill slots 0 and 1 (as the oracle orders them),
+    slots 2 and 3 get id 0x7fffffff and gate 0 (GEMM mode: gate 0 too), add no
+    load, and EBL_ST_NONFINITE is raised.  A finite bias raises nothing."""
+    dev = cuda_device
+    T, Nr, K, d = 300, 64, 4, 128
+    live = [5, 40]
+    bias = torch.full((Nr,), float("-inf"))
+    bias[live] = 0.0
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    if mode == "gemm":
+        h = synth.hidden_normal(T, d, seed=61)
+        W = synth.router_weight(Nr, d, seed=62)
+        idx, g = ebl.router_forward(h.to(dev), W.to(dev), bias.to(dev), K, counts, status=st)
+        ref = oracle.router_gemm(h, W, np.zeros(Nr, np.float32), K, want_scores=True)
+        scores = ref.scores
+    else:
+        x = synth.logits_normal(T, Nr, seed=63)
+        if mode == "logits_row":               # 4 bytes past a 16-byte boundary: the row kernel
+            buf = torch.empty(T * Nr + 1, device=dev)
+            buf[1:] = x.reshape(-1).to(dev)
+            xd = buf[1:].view(T, Nr)
+        else:
+            xd = x.to(dev)
+        idx, g = ebl.router_forward_logits(xd, bias.to(dev), K, counts, status=st)
+        scores = oracle.router_logits(x.numpy(), np.zeros(Nr, np.float32), 1, want_scores=True).scores
+    torch.cuda.synchronize()
+    assert int(st.item()) == ebl.EBL_ST_NONFINITE
+    gi, gg = to_np(idx), to_np(g)
+    s = scores[:, live]
+    first = np.where(s[:, 0] >= s[:, 1], live[0], live[1])   # equal scores: the lower index first
+    second = np.where(first == live[0], live[1], live[0])
+    # GEMM mode orders the two the oracle's way except where fp32 and fp64
+    # scores may disagree (keys closer than the near-tie margin)
+    rows = np.abs(s[:, 0] - s[:, 1]) >= (1e-3 if mode == "gemm" else 0.0)
+    assert rows.sum() > T // 2
+    assert np.array_equal(gi[rows, 0], first[rows]) and np.array_equal(gi[rows, 1], second[rows])
+    assert np.all(np.sort(gi[:, :2], 1) == np.array(live))
+    assert np.all(gi[:, 2:] == 0x7fffffff)
+    assert np.all(gg[:, 2:] == 0.0)
+    assert np.allclose(gg[:, :2].sum(1), 1.0, atol=1e-6)
+    c = to_np(counts)
+    assert c[live].sum() == 2 * T and c.sum() == 2 * T
+
+    # finite bias: nothing raised
+    st.zero_()
+    counts.zero_()
+    if mode == "gemm":
+        ebl.router_forward(h.to(dev), W.to(dev), torch.zeros(Nr, device=dev), K, counts, status=st)
+    else:
+        ebl.router_forward_logits(xd, torch.zeros(Nr, device=dev), K, counts, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0

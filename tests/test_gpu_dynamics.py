@@ -1,47 +1,86 @@
-"""Multi-step balancing runs on the mid and drift workloads (GEMM mode, full
-size) and a CUDA-graph capture of the router step.
+"""Multi-step balancing runs on the full-size workloads and CUDA-graph
+captures of the router step.
+
+Every multi-step run is checked open loop against the oracle ("SMEBU Load
+Balancing", "How it works", eqs. (20)-(28)): each step the oracle's update is
+fed the loads the library's router produced and must leave the same bias and
+momentum (within 1e-6 relative, floor 1e-9) as the library's update, step by
+step.  The routing itself is checked each step on sampled rows against the
+oracle's fp64 router with the same bias (the GEMM-mode near-tie rule).  The
+logits-mode closed loop on the full tie workload is bit-exact in the loads, so
+there the oracle routes every token with its own bias and both trajectories
+must agree.
 
 The pages give no numbers for the dynamics (SMEBU settles, the sign update
-keeps oscillating at +-gamma, a linear update goes unstable), so these tests
-assert only what the equations fix -- sum of b stays at its start value under
-SMEBU (the step is re-centred) and at 0 under the sign update (b is
+keeps oscillating at +-gamma, a linear update goes unstable), so beyond parity
+these tests assert only what the equations fix -- sum of b stays at its start
+value under SMEBU (the step is re-centred) and at 0 under the sign update (b is
 re-centred), |m| <= 2 lambda, the loads add up to K*T -- and print the MaxVio
 trajectories (pytest -s) as the workloads ask.
 """
 import json
 import math
 
+import numpy as np
 import pytest
 import torch
 
 import expert_bias_load_b200 as ebl
+import oracle
 import synth
 from expert_bias_load_b200.telemetry import maxvio_level, step_stats
+from tests.parity import STATE_RTOL, assert_gemm_parity, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
+SAMPLE_ROWS = 256     # rows per step checked against the oracle's fp64 router
 
-def _run(h_of_step, W, K, steps, update, gamma=1e-3):
+
+def _run(h_of_step, W, K, steps, update, gamma=1e-3, b0=None, sample_rows=SAMPLE_ROWS, seed=0):
+    """Route a fresh batch each step and apply the bias update; alongside, the
+    oracle's update takes the library's loads of the same step (open loop) and
+    its state must match the library's at every step."""
     dev = W.device
     Nr = W.shape[0]
-    b = torch.zeros(Nr, device=dev)
+    b = torch.zeros(Nr, device=dev) if b0 is None else b0.to(dev).clone()
     m = torch.zeros(Nr, device=dev)
+    b_o = to_np(b).copy()
+    m_o = np.zeros(Nr, np.float32)
+    W_cpu = W.cpu()
+    rng = np.random.default_rng(seed)
     counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
     mv = torch.zeros(1, device=dev)
     traj = []
+    worst = [0.0, 0.0]
     for s in range(steps):
         h = h_of_step(s)
-        ebl.router_forward(h, W, b, K, counts)
+        T = h.shape[0]
+        idx, g = ebl.router_forward(h, W, b, K, counts)
         prev = b.clone()
         c = counts.clone()
+        if sample_rows:
+            rows = np.sort(rng.choice(T, size=min(sample_rows, T), replace=False))
+            rt = torch.from_numpy(rows).to(dev)
+            bias_used = to_np(prev)
+            ref = oracle.router_gemm(h.index_select(0, rt).cpu(), W_cpu, bias_used, K, want_scores=True)
+            assert_gemm_parity(to_np(idx.index_select(0, rt)), to_np(g.index_select(0, rt)), ref, Nr, bias_used)
+        n = to_np(c).astype(np.int64)
         if update == "smebu":
             ebl.smebu_step(counts, b, m, reset_counts=True, maxvio=mv)
+            _, mvo = oracle.smebu(n, b_o, m_o)
         else:
             ebl.sign_update_step(counts, b, gamma, reset_counts=True, maxvio=mv)
+            _, mvo = oracle.sign_update(n, b_o, gamma)
+        eb = float(rel_err(to_np(b), b_o).max())
+        em = float(rel_err(to_np(m), m_o).max())
+        assert eb <= STATE_RTOL and em <= STATE_RTOL, (update, s, eb, em)
+        worst = [max(worst[0], eb), max(worst[1], em)]
+        g_mv = float(mv.item())
+        assert g_mv == mvo or (math.isinf(g_mv) and math.isinf(mvo)), (s, g_mv, mvo)
         st = step_stats(c, b, m if update == "smebu" else None, mv, prev)
-        assert st["total_load"] == K * h.shape[0]
+        assert st["total_load"] == K * T
         traj.append(st)
-    return traj, b, m
+    return traj, b, m, worst
 
 
 def test_mid_workload_sign_vs_smebu(cuda_device):
@@ -49,15 +88,15 @@ def test_mid_workload_sign_vs_smebu(cuda_device):
     T, d, Nr, K, steps = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"], cfg["steps"]
     W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(cuda_device)
     hs = lambda s: synth.hidden_normal(T, d, seed=synth.step_seed("mid", s), device=cuda_device)
-    tr_smebu, b1, m1 = _run(hs, W, K, steps, "smebu")
-    tr_sign, b2, _ = _run(hs, W, K, steps, "sign")
+    tr_smebu, b1, m1, w1 = _run(hs, W, K, steps, "smebu", seed=1)
+    tr_sign, b2, _, w2 = _run(hs, W, K, steps, "sign", seed=2)
     for st in tr_smebu:
         assert abs(st["bias_sum"]) <= 1e-4                   # b0 = 0 and every step sums to 0
         assert st["momentum_absmax"] <= 2 * 5e-4 * (1 + 1e-6)
     for st in tr_sign:
         assert abs(st["bias_sum"]) <= 1e-4                   # b is re-centred every step
         assert st["bias_step_absmax"] <= 2 * 1e-3 * (1 + 1e-6)
-    print("\nmid workload MaxVio per step")
+    print("\nmid workload MaxVio per step; worst relative state error vs the oracle: smebu %s, sign %s" % (w1, w2))
     print(json.dumps({"smebu": [round(s["maxvio"], 3) for s in tr_smebu],
                       "sign": [round(s["maxvio"], 3) for s in tr_sign]}))
 
@@ -80,13 +119,68 @@ def test_drift_workload_smebu_200_steps(cuda_device):
             break
     assert mu is not None, "no drift strength on the scan gives MaxVio > 6"
     hs = lambda s: synth.hidden_drift(T, d, W, seed=synth.step_seed("drift", s), mu=mu, device=dev)
-    tr, b, m = _run(hs, W, K, steps, "smebu")
+    tr, b, m, worst = _run(hs, W, K, steps, "smebu", seed=3)
     assert maxvio_level(tr[0]["maxvio"]) == "alarm"
     for st in tr:
         assert abs(st["bias_sum"]) <= 1e-4
         assert st["momentum_absmax"] <= 2 * 5e-4 * (1 + 1e-6)
-    print("\ndrift workload mu=%g MaxVio every 10 steps" % mu)
+    print("\ndrift workload mu=%g MaxVio every 10 steps; worst relative state error vs the oracle %s" % (mu, worst))
     print(json.dumps([round(tr[i]["maxvio"], 3) for i in range(0, steps, 10)] + [round(tr[-1]["maxvio"], 3)]))
+
+
+def test_tie_workload_gemm_smebu_100_steps(cuda_device):
+    """The tie workload in GEMM mode at full size (T = 1,048,576, d = 4096,
+    N_r = 256, K = 4, hidden on the 1/8 grid, 8 experts starting at bias
+    -1.0): 100 SMEBU steps, open loop against the oracle every step."""
+    cfg = synth.WORKLOADS["ties"]
+    T, d, Nr, K, steps = cfg["T"], cfg["d"], cfg["Nr"], cfg["K"], cfg["steps"]
+    dev = cuda_device
+    W = synth.router_weight(Nr, d, seed=synth.BASE_SEED + d).to(dev)
+    hs = lambda s: synth.hidden_normal(T, d, seed=synth.step_seed("ties", s), device=dev, quant8=True)
+    tr, b, m, worst = _run(hs, W, K, steps, "smebu", b0=synth.dead_start_bias(Nr), seed=5)
+    assert math.isinf(tr[0]["maxvio"])                # the dead-start experts get no load at step 0
+    for st in tr:
+        assert abs(st["bias_sum"] - (-8.0)) <= 1e-4  # sum of b stays at its start value
+        assert st["momentum_absmax"] <= 2 * 5e-4 * (1 + 1e-6)
+    print("\ntie workload (GEMM) MaxVio every 10 steps; worst relative state error vs the oracle %s" % (worst,))
+    print(json.dumps([round(tr[i]["maxvio"], 3) for i in range(0, steps, 10)] + [round(tr[-1]["maxvio"], 3)]))
+
+
+def test_tie_workload_logits_closed_loop_full_size(cuda_device):
+    """Logits mode on the full tie workload (T = 1,048,576 tokens of fp32
+    logits on the 1/8 grid, N_r = 256, K = 4, dead start): 100 SMEBU steps in
+    closed loop on both sides -- the library and the oracle each route every
+    token with their own bias and update it from their own loads.  Loads are
+    bit-exact, so the indices, gates and loads must be identical every step
+    and the state within 1e-6 relative."""
+    cfg = synth.WORKLOADS["ties"]
+    T, Nr, K, steps = cfg["T"], cfg["Nr"], cfg["K"], cfg["steps"]
+    dev = cuda_device
+    b_g = synth.dead_start_bias(Nr, device=dev)
+    m_g = torch.zeros(Nr, device=dev)
+    b_o = synth.dead_start_bias(Nr).numpy()
+    m_o = np.zeros(Nr, np.float32)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    g = torch.empty(T, K, device=dev)
+    mv = torch.zeros(1, device=dev)
+    mvs = []
+    for s in range(steps):
+        x = synth.logits_normal(T, Nr, seed=synth.step_seed("ties", s), device=dev, quant8=True)
+        ebl.router_forward_logits(x, b_g, K, counts, topk_idx=idx, gates=g)
+        ref = oracle.router_logits(to_np(x), b_o, K)
+        del x
+        assert np.array_equal(to_np(counts).astype(np.int64), ref.counts), s
+        assert np.array_equal(to_np(idx), ref.idx), s
+        assert np.array_equal(to_np(g), ref.gates), s
+        ebl.smebu_step(counts, b_g, m_g, reset_counts=True, maxvio=mv)
+        oracle.smebu(ref.counts, b_o, m_o)
+        assert rel_err(to_np(b_g), b_o).max() <= STATE_RTOL, s
+        assert rel_err(to_np(m_g), m_o).max() <= STATE_RTOL, s
+        mvs.append(float(mv.item()))
+    assert math.isinf(mvs[0])
+    print("\ntie workload (logits, closed loop) MaxVio every 10 steps")
+    print(json.dumps([round(mvs[i], 3) for i in range(0, steps, 10)] + [round(mvs[-1], 3)]))
 
 
 def test_router_step_in_cuda_graph(cuda_device):

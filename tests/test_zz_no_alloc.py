@@ -7,16 +7,22 @@ keeps the scratch in a fixed library-owned device array instead.  The test
 calls it through the C ABI twice in a row, on different inputs, and checks each
 result against moe_dispatch with a caller workspace: offsets, perm, dest and
 the gathered rows must be identical (dispatch is exact integer and copy work).
-It also checks that a problem too large for the array is refused.
+Each result is also checked on its own against the oracle's stable expert sort
+(offsets, perm, dest) and against the rows of hidden it names.  One case passes
+no status word, so device-side errors would go to the library's own word; it
+must still give the same outputs.  A problem too large for the array is
+refused.
 
 The file name makes pytest collect it last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
 import expert_bias_load_b200 as ebl
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -48,8 +54,8 @@ def _static_dispatch(hidden, idx, Nr, tile_counts, status, stream):
     return rc, offsets, perm, dest, X
 
 
-@pytest.mark.parametrize("with_tiles", [False, True])
-def test_static_dispatch_matches_workspace_dispatch_twice(cuda_device, with_tiles):
+@pytest.mark.parametrize("with_tiles,with_status", [(False, True), (True, True), (True, False)])
+def test_static_dispatch_matches_workspace_dispatch_twice(cuda_device, with_tiles, with_status):
     dev = cuda_device
     stream = torch.cuda.current_stream()
     # two calls in a row on different problems; the second must not see the first's scratch
@@ -60,16 +66,23 @@ def test_static_dispatch_matches_workspace_dispatch_twice(cuda_device, with_tile
         if with_tiles:
             tiles = torch.stack([torch.bincount(idx[j * 128:(j + 1) * 128].reshape(-1).long(), minlength=Nr)
                                  for j in range((T + 127) // 128)]).to(torch.int32)
-        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev) if with_status else None
         rc, offsets, perm, dest, X = _static_dispatch(h, idx, Nr, tiles, st, stream)
         assert rc == 0, ebl.lib().ebl_strerror(rc)
         ref = ebl.moe_dispatch(h, idx, Nr, tile_counts=tiles)
         torch.cuda.synchronize()
-        assert int(st.item()) == 0
+        if with_status:
+            assert int(st.item()) == 0
         assert torch.equal(offsets, ref[0])
         assert torch.equal(perm, ref[1])
         assert torch.equal(dest, ref[2])
         assert torch.equal(X, ref[3])
+        # independent of the other entry point: the oracle's stable expert sort
+        o_off, o_perm, o_dest = oracle.dispatch(idx.cpu().numpy(), Nr)
+        assert np.array_equal(offsets.cpu().numpy(), o_off)
+        assert np.array_equal(perm.cpu().numpy(), o_perm)
+        assert np.array_equal(dest.cpu().numpy(), o_dest)
+        assert torch.equal(X, h[perm.long()])
 
 
 def test_static_dispatch_rejects_oversized_problem(cuda_device):
