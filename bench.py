@@ -637,15 +637,29 @@ def main():
         extra["logits_mode"] = {"tokens_per_s": T * world / (lm / 1e3), "ms": lm,
                                 "achieved_gbs": lbytes / (lm / 1e3) / 1e9,
                                 "frac_hbm": lbytes / (lm / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        # the balance statistics fused into the routing pass (one read of the
+        # logits), and as the separate fp64 pass
         tpl = torch.empty((T + 127) // 128, Nr, dtype=torch.float32, device=dev)
+        tcl = torch.empty((T + 127) // 128, Nr, dtype=torch.int32, device=dev)
+        for _ in range(2):
+            ebl.router_forward_logits_balance(x, bias, K, counts, tcl, tpl, topk_idx=idx, gates=gates, stream=stream)
+        counts.zero_()
+        ev[0].record(stream)
+        for _ in range(reps):
+            ebl.router_forward_logits_balance(x, bias, K, counts, tcl, tpl, topk_idx=idx, gates=gates, stream=stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        fm = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
+        extra["logits_mode"]["fused_balance_ms"] = fm
+        extra["logits_mode"]["balance_stats_ms"] = fm - lm
         ebl.balance_stats_logits(x, tile_psum=tpl, stream=stream)
         ev[0].record(stream)
         for _ in range(reps):
             ebl.balance_stats_logits(x, tile_psum=tpl, stream=stream)
         ev[1].record(stream)
         torch.cuda.synchronize()
-        extra["logits_mode"]["balance_stats_ms"] = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
-        del tpl
+        extra["logits_mode"]["balance_stats_separate_fp64_ms"] = max_over_ranks([ev[0].elapsed_time(ev[1]) / reps])[0]
+        del tpl, tcl
         counts.zero_()
         del x
 

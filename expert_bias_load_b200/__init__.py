@@ -22,7 +22,8 @@ import torch
 
 __all__ = [
     "EblError", "lib", "lib_path", "tile_tokens", "router_forward", "router_forward_zloss", "router_forward_balance",
-    "seq_balance_loss", "balance_stats_logits", "router_forward_logits", "smebu_step",
+    "seq_balance_loss", "balance_stats_logits", "router_forward_logits", "router_forward_logits_balance",
+    "smebu_step",
     "smebu_step_layers", "sign_update_step", "moe_dispatch", "moe_combine", "dispatch_workspace_bytes",
     "read_internal_status", "check_finite", "EBL_ST_BAD_EXPERT", "EBL_ST_BAD_DEST", "EBL_ST_EMPTY_LOAD",
     "EBL_ST_TIMEOUT", "EBL_ST_BAD_COUNTS", "EBL_ST_NONFINITE",
@@ -55,6 +56,7 @@ SIGNATURES = {
     "router_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "router_forward_zloss": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "router_forward_logits": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "router_forward_logits_balance": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "router_forward_balance": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "seq_balance_loss": (_I, [_P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "balance_stats_logits": (_I, [_P, _I, _I, _P, _P]),
@@ -263,6 +265,26 @@ def router_forward_logits(logits, bias, K, counts, topk_idx=None, gates=None, ti
         _check(tile_counts, "tile_counts", torch.int32, ((T + 127) // 128, Nr))
     _call("router_forward_logits", _ptr(logits), _ptr(bias), T, Nr, K, _ptr(topk_idx), _ptr(gates),
           _ptr(counts), _ptr(tile_counts), _ptr(status), _stream(stream))
+    return topk_idx, gates
+
+
+def router_forward_logits_balance(logits, bias, K, counts, tile_counts, tile_psum, topk_idx=None, gates=None,
+                                  status=None, stream=None):
+    """router_forward_logits that also writes the per-tile statistics of the
+    sequence-wise balance loss in the same pass over the logits: tile_counts
+    int32 and tile_psum fp32, both [ceil(T/128), N_r].  Returns (topk_idx, gates)."""
+    _check(logits, "logits", torch.float32)
+    T, Nr = logits.shape
+    _check(bias, "bias", torch.float32, (Nr,))
+    _check(counts, "counts", torch.int32, (Nr,))
+    tiles = (T + 127) // 128
+    _check(tile_counts, "tile_counts", torch.int32, (tiles, Nr))
+    _check(tile_psum, "tile_psum", torch.float32, (tiles, Nr))
+    dev = logits.device
+    topk_idx = _out(topk_idx, "topk_idx", (T, K), torch.int32, dev)
+    gates = _out(gates, "gates", (T, K), torch.float32, dev)
+    _call("router_forward_logits_balance", _ptr(logits), _ptr(bias), T, Nr, K, _ptr(topk_idx), _ptr(gates),
+          _ptr(counts), _ptr(tile_counts), _ptr(tile_psum), _ptr(status), _stream(stream))
     return topk_idx, gates
 
 

@@ -233,9 +233,36 @@ int router_forward_logits(const float *logits, const float *bias, int T, int N_r
     DeviceInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
-    cudaError_t e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts,
+    cudaError_t e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts, nullptr,
                                               status ? status : di.internal_status, di.num_sms,
                                               reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
+}
+
+int router_forward_logits_balance(const float *logits, const float *bias, int T, int N_r, int K, int32_t *topk_idx,
+                                  float *gates, int32_t *counts, int32_t *tile_counts, float *tile_psum,
+                                  int32_t *status, ebl_stream_t stream) {
+    if (check_T(T) || check_topk(N_r, K)) return EBL_EINVAL;
+    if (!bias || !counts) return EBL_EINVAL;
+    if (T > 0 && (!logits || !topk_idx || !gates || !tile_counts || !tile_psum)) return EBL_EINVAL;
+    if (!aligned4(logits) || !aligned4(bias) || !aligned4(topk_idx) || !aligned4(gates) || !aligned4(counts) ||
+        !aligned4(tile_counts) || !aligned4(tile_psum))
+        return EBL_EINVAL;
+    if (T == 0) return EBL_OK;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t *stw = status ? status : di.internal_status;
+    cudaError_t e;
+    if (ebl::logits_vector_path(logits, N_r)) {
+        e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts, tile_psum, stw,
+                                      di.num_sms, st);
+    } else {  // any N_r and alignment: the row kernel, then the balance statistics as their own pass
+        e = ebl::launch_router_logits(logits, bias, T, N_r, K, topk_idx, gates, counts, tile_counts, nullptr, stw,
+                                      di.num_sms, st);
+        if (e == cudaSuccess) e = ebl::launch_tile_psum_logits(logits, T, N_r, tile_psum, di.num_sms, st);
+    }
     return e == cudaSuccess ? EBL_OK : cuda_fail("kernel launch", e);
 }
 

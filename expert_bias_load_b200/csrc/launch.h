@@ -22,9 +22,11 @@ cudaError_t launch_router_gemm(const CUtensorMap &tmap_h, const CUtensorMap &tma
                                int num_sms, cudaStream_t stream);
 
 // router_logits.cu
+// tile_psum != NULL (the balance option) needs the vector path: logits_vector_path()
+bool logits_vector_path(const float *logits, int Nr);
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
-                                 float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms,
-                                 cudaStream_t stream);
+                                 float *gates, int32_t *counts, int32_t *tile_counts, float *tile_psum,
+                                 int32_t *status, int num_sms, cudaStream_t stream);
 cudaError_t launch_score_error(const float *x, int64_t n, float *max_err, float *exact_out, cudaStream_t stream);
 cudaError_t launch_check_finite(const void *p, int64_t n, int bf16, int32_t *status, int num_sms,
                                 cudaStream_t stream);

@@ -249,8 +249,8 @@ __device__ __forceinline__ float key_approx(float x, float hb) { return fmaf(0.5
 // rounding of this fp32 expression) key_a >= tau' - 2 kKeyErr - 2^-19 |tau'|.
 // An empty list (tau' = -inf) admits every finite key; padding keys (-inf)
 // never pass.
-__device__ __forceinline__ float candidate_limit(float tau) {
-    return fmaxf(tau - (2.0f * kKeyErr + 0x1p-19f * fabsf(tau)), -FLT_MAX);
+__device__ __forceinline__ float candidate_limit(float tau, float key_err = kKeyErr) {
+    return fmaxf(tau - (2.0f * key_err + 0x1p-19f * fabsf(tau)), -FLT_MAX);
 }
 
 constexpr int kStages = 2;  // row groups of a warp in the shared-memory ring: one loads while one is ranked
@@ -272,27 +272,46 @@ constexpr size_t vec_ring_bytes() {
     return sizeof(float) * kWarpsPerCta * kStages * kRowsPerGroup * 32 * NV;
 }
 
-template <int K, int NV, bool FULL>
+// Per-warp candidate buffers of the vector kernel.  With the balance option a
+// warp's column sums (kMaxExperts floats) reuse this space at the end of each
+// tile, after the warp's last candidate stage of the tile.
+struct WarpCand {
+    int c[kRowsPerGroup][kWinPad];  // a round's candidates of each row
+    float key[kRowsPerGroup][kWinPad];
+    float s[kRowsPerGroup][kWinPad];
+};
+static_assert(sizeof(WarpCand) >= kMaxExperts * sizeof(float), "column sums fit the candidate buffers");
+
+// BAL (the balance option): the approximate key is sigmoid_fast(x) + b instead
+// of the tanh form, and the same fast scores give the per-tile statistics of
+// the sequence-wise balance loss, tile_psum[j, i] = sum over the tile's rows t
+// of s_t,i / sum_l s_t,l.  Each lane keeps the fp32 sums of its 4*NV columns
+// over the rows it sees; at the end of a tile the warp folds its four row
+// lanes per column with two shuffles and the CTA adds its four warps in
+// order, so the sums do not depend on scheduling.
+template <int K, int NV, bool FULL, bool BAL>
 __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float *__restrict__ logits,
                                                                      const float *__restrict__ bias, int T, int Nr,
                                                                      int32_t *__restrict__ topk_idx,
                                                                      float *__restrict__ gates,
                                                                      int32_t *__restrict__ counts,
                                                                      int32_t *__restrict__ tile_counts,
+                                                                     float *__restrict__ tile_psum,
                                                                      int32_t *__restrict__ status) {
     // lane-local lists of the approximate pass hold P >= K values (P a power of two)
     constexpr int P = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
     constexpr int kRow = 32 * NV;  // floats per row in the ring (N_r rounded up, zero-filled)
     // FULL: N_r == kRow, so every column a lane copies exists (no per-column test)
     static_assert(NV % 2 == 0 && kRow <= kMaxExperts, "a lane holds NV float4 of a row, in pairs");
+    // distance of the approximate key to the exact one (see key_approx, sigmoid_fast)
+    constexpr float kErr = BAL ? kSigmaErr : kKeyErr;
     extern __shared__ __align__(16) float ring_s[];  // [warp][stage][row of group][kRow]
-    __shared__ __align__(16) float hb_s[kMaxExperts];  // fl(0.5 + b); -inf past N_r
+    // tanh form: fl(0.5 + b); balance option: b.  -inf past N_r either way.
+    __shared__ __align__(16) float hb_s[kMaxExperts];
     __shared__ float bias_s[kMaxExperts];
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
-    __shared__ int cand_c[kWarpsPerCta][kRowsPerGroup][kWinPad];  // a round's candidates of each row
-    __shared__ float cand_key[kWarpsPerCta][kRowsPerGroup][kWinPad];
-    __shared__ float cand_s[kWarpsPerCta][kRowsPerGroup][kWinPad];
+    __shared__ __align__(16) WarpCand cand[kWarpsPerCta];
     __shared__ float sel_key[kWarpsPerCta][kRowsPerGroup][2 * K];  // [0,K): the Top-K so far; [K,2K): a later round's
     __shared__ float sel_s[kWarpsPerCta][kRowsPerGroup][2 * K];
     __shared__ int sel_c[kWarpsPerCta][kRowsPerGroup][2 * K];
@@ -301,7 +320,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         const bool in = i < Nr;
         const float b = in ? bias[i] : 0.0f;
         bias_s[i] = b;
-        hb_s[i] = in ? __fadd_rn(0.5f, b) : -INFINITY;
+        hb_s[i] = in ? (BAL ? b : __fadd_rn(0.5f, b)) : -INFINITY;
         hist_total[i] = 0;
         hist_tile[i] = 0;
     }
@@ -320,9 +339,10 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     const int r = lane >> 3;  // row of the group this lane works on
     const int j = lane & 7;   // lane within the row: float4 columns j, j + 8, j + 16, ...
     float *ring = ring_s + (size_t)warp * kStages * kRowsPerGroup * kRow;
-    int *cc = cand_c[warp][r];
-    float *ck = cand_key[warp][r];
-    float *cs = cand_s[warp][r];
+    int *cc = cand[warp].c[r];
+    float *ck = cand[warp].key[r];
+    float *cs = cand[warp].s[r];
+    float *colsum = reinterpret_cast<float *>(&cand[warp]);  // balance option: the warp's column sums
     float *sk = sel_key[warp][r];
     float *ss = sel_s[warp][r];
     int *sc = sel_c[warp][r];
@@ -357,6 +377,11 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                           ? ((num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * kGroupsPerWarp
                           : 0;
     static_assert(kStages == 2, "one item in flight while one is ranked");
+    float psum[BAL ? NV : 1][4];  // balance option: this lane's column sums over the tile's rows it sees
+#pragma unroll
+    for (int m = 0; m < (BAL ? NV : 1); ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) psum[m][e] = 0.0f;
     int64_t ahead = item_row(0);  // the row of the most recently issued item
     issue(0, ahead);
     for (int item = 0; item < items; ++item) {
@@ -369,14 +394,48 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
 
         // approximate keys of this lane's 4*NV experts
         float kv[NV][4];
+        if constexpr (BAL) {
+            // fast scores; their row total over the row's 8 lanes; the lane's
+            // column sums gain s / total (0 for a row past T); then the keys
+            float rs = 0.0f;
 #pragma unroll
-        for (int m = 0; m < NV; ++m) {
-            const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
-            const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
-            kv[m][0] = key_approx(x.x, h.x);
-            kv[m][1] = key_approx(x.y, h.y);
-            kv[m][2] = key_approx(x.z, h.z);
-            kv[m][3] = key_approx(x.w, h.w);
+            for (int m = 0; m < NV; ++m) {
+                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
+                kv[m][0] = sigmoid_fast(x.x);
+                kv[m][1] = sigmoid_fast(x.y);
+                kv[m][2] = sigmoid_fast(x.z);
+                kv[m][3] = sigmoid_fast(x.w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if constexpr (!FULL)  // padding columns (zero-filled, s = 1/2) add nothing
+                        if (4 * (8 * m + j) + e >= Nr) kv[m][e] = 0.0f;
+                    rs += kv[m][e];
+                }
+            }
+            rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+            rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+            rs += __shfl_xor_sync(0xffffffffu, rs, 4);
+            const float inv = (row < T && rs > 0.0f) ? __frcp_rn(rs) : 0.0f;
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
+                const float hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    psum[m][e] = fmaf(kv[m][e], inv, psum[m][e]);
+                    kv[m][e] = __fadd_rn(kv[m][e], hv[e]);  // -inf past N_r
+                }
+            }
+        } else {
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
+                const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
+                kv[m][0] = key_approx(x.x, h.x);
+                kv[m][1] = key_approx(x.y, h.y);
+                kv[m][2] = key_approx(x.z, h.z);
+                kv[m][3] = key_approx(x.w, h.w);
+            }
         }
         // tau': the K-th largest of the maxima of groups of 8 keys (each
         // maximum is a key of its own, so tau' is at most the K-th key)
@@ -415,7 +474,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         top.merge_xor(1);
         top.merge_xor(2);
         top.merge_xor(4);
-        const float lim = candidate_limit(top.v[K - 1]);
+        const float lim = candidate_limit(top.v[K - 1], kErr);
         unsigned mask = 0;
 #pragma unroll
         for (int m = 0; m < NV; ++m)
@@ -567,12 +626,33 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
 
         if (want_tiles && (item & 7) == 7) {
             const int tile = (int)blockIdx.x + (item >> 3) * (int)gridDim.x;
+            if constexpr (BAL) {
+                // the warp's 32 rows per column: lanes j, j + 8, j + 16, j + 24
+                // hold the same columns; fold them (fixed order), lanes 0..7 store
+#pragma unroll
+                for (int m = 0; m < NV; ++m)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float v = psum[m][e];
+                        v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        if (r == 0) colsum[4 * (8 * m + j) + e] = v;
+                        psum[m][e] = 0.0f;
+                    }
+            }
             __syncthreads();
             for (int e = threadIdx.x; e < Nr; e += kThreads) {
                 const int v = hist_tile[e];
                 tile_counts[(size_t)tile * Nr + e] = v;
                 hist_total[e] += v;
                 hist_tile[e] = 0;
+                if constexpr (BAL) {
+                    const float *c0 = reinterpret_cast<const float *>(&cand[0]);
+                    const float *c1 = reinterpret_cast<const float *>(&cand[1]);
+                    const float *c2 = reinterpret_cast<const float *>(&cand[2]);
+                    const float *c3 = reinterpret_cast<const float *>(&cand[3]);
+                    tile_psum[(size_t)tile * Nr + e] = ((c0[e] + c1[e]) + c2[e]) + c3[e];
+                }
             }
             __syncthreads();
         }
@@ -632,10 +712,11 @@ cudaError_t vec_setup(const void *kern, size_t smem, int *blocks_per_sm) {
     return cudaSuccess;
 }
 
-template <int K, int NV, bool FULL>
+template <int K, int NV, bool FULL, bool BAL>
 cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, int32_t *topk_idx, float *gates,
-                       int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms, cudaStream_t stream) {
-    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL>);
+                       int32_t *counts, int32_t *tile_counts, float *tile_psum, int32_t *status, int num_sms,
+                       cudaStream_t stream) {
+    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL, BAL>);
     const size_t smem = vec_ring_bytes<NV>();
     int per_sm = 1;
     cudaError_t err = vec_setup(kern, smem, &per_sm);
@@ -643,26 +724,33 @@ cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, in
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     int grid = num_sms * per_sm;
     if (grid > num_tiles) grid = num_tiles;
-    router_logits_vec_kernel<K, NV, FULL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates,
-                                                                            counts, tile_counts, status);
+    router_logits_vec_kernel<K, NV, FULL, BAL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx,
+                                                                                 gates, counts, tile_counts,
+                                                                                 tile_psum, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+bool logits_vector_path(const float *logits, int Nr) {
+    return Nr % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+}
+
 cudaError_t launch_router_logits(const float *logits, const float *bias, int T, int Nr, int K, int32_t *topk_idx,
-                                 float *gates, int32_t *counts, int32_t *tile_counts, int32_t *status, int num_sms,
-                                 cudaStream_t stream) {
+                                 float *gates, int32_t *counts, int32_t *tile_counts, float *tile_psum,
+                                 int32_t *status, int num_sms, cudaStream_t stream) {
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
-    if (Nr % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15) == 0) {
+    if (logits_vector_path(logits, Nr)) {
         // vector kernel: persistent CTAs, as many per SM as fit
         const int nv = Nr <= 64 ? 2 : (Nr <= 128 ? 4 : 8);
+        const bool bal = tile_psum != nullptr;
         switch (K * 16 + nv) {
-#define EBL_VCASE(KK, NN) \
-    case KK * 16 + NN:    \
-        return Nr == 32 * NN                                                                                   \
-                   ? launch_vec<KK, NN, true>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, status, num_sms, stream) \
-                   : launch_vec<KK, NN, false>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, status, num_sms, stream);
+#define EBL_VLAUNCH(KK, NN, F, B) \
+    launch_vec<KK, NN, F, B>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, tile_psum, status, num_sms, stream)
+#define EBL_VCASE(KK, NN)                                                                          \
+    case KK * 16 + NN:                                                                             \
+        if (bal) return Nr == 32 * NN ? EBL_VLAUNCH(KK, NN, true, true) : EBL_VLAUNCH(KK, NN, false, true); \
+        return Nr == 32 * NN ? EBL_VLAUNCH(KK, NN, true, false) : EBL_VLAUNCH(KK, NN, false, false);
 #define EBL_VCASES(KK) EBL_VCASE(KK, 2) EBL_VCASE(KK, 4) EBL_VCASE(KK, 8)
             EBL_VCASES(1)
             EBL_VCASES(2)
@@ -674,11 +762,14 @@ cudaError_t launch_router_logits(const float *logits, const float *bias, int T, 
             EBL_VCASES(8)
 #undef EBL_VCASES
 #undef EBL_VCASE
+#undef EBL_VLAUNCH
             default:
                 return cudaErrorInvalidValue;
         }
     }
-    // row kernel: any N_r and alignment
+    // row kernel: any N_r and alignment (the balance option runs beside it, as a
+    // separate pass: launch_tile_psum_logits)
+    if (tile_psum) return cudaErrorInvalidValue;
     int grid = num_sms * 16;
     if (grid > num_tiles) grid = num_tiles;
     switch (K) {

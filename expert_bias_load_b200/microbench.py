@@ -12,7 +12,9 @@ public binding, so it is also the command to put under a profiler: with
 Entry points: router (GEMM mode), zloss (GEMM mode with the z-loss), balance
 (GEMM mode with the sequence-wise balance statistics, then the loss over
 sequences of 4096 tokens, or of T tokens when T is smaller), logits (logits
-mode), balance_logits (the logits-mode balance statistics), smebu, sign,
+mode), logits_balance (logits mode with the balance statistics in the same
+pass), balance_logits (the logits-mode balance statistics as a separate fp64
+pass), smebu, sign,
 dispatch, combine.  For the one-CTA update kernels
 (smebu, sign) the time per call is the host's launch rate, not the kernel's.
 """
@@ -41,8 +43,8 @@ def _time(fn, warmup, reps):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("op", choices=["router", "zloss", "balance", "logits", "balance_logits", "smebu", "sign", "dispatch",
-                                   "combine"])
+    ap.add_argument("op", choices=["router", "zloss", "balance", "logits", "logits_balance", "balance_logits", "smebu",
+                                   "sign", "dispatch", "combine"])
     ap.add_argument("--tokens", type=int, default=1 << 20)
     ap.add_argument("--hidden", type=int, default=4096)
     ap.add_argument("--experts", type=int, default=256)
@@ -86,6 +88,15 @@ def main(argv=None):
         idx = torch.empty(T, K, dtype=torch.int32, device=dev)
         g = torch.empty(T, K, device=dev)
         fn = lambda: ebl.router_forward_logits(x, bias, K, counts, topk_idx=idx, gates=g)
+        ms = _time(fn, a.warmup, a.reps)
+        work = "%.1f GB/s" % ((T * Nr * 4 + T * K * 8) / ms / 1e6)
+    elif a.op == "logits_balance":
+        x = synth.logits_normal(T, Nr, seed=a.seed, device=dev, quant8=True)
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        g = torch.empty(T, K, device=dev)
+        tc = torch.empty((T + 127) // 128, Nr, dtype=torch.int32, device=dev)
+        tp = torch.empty((T + 127) // 128, Nr, device=dev)
+        fn = lambda: ebl.router_forward_logits_balance(x, bias, K, counts, tc, tp, topk_idx=idx, gates=g)
         ms = _time(fn, a.warmup, a.reps)
         work = "%.1f GB/s" % ((T * Nr * 4 + T * K * 8) / ms / 1e6)
     elif a.op == "balance_logits":

@@ -236,6 +236,32 @@ int router_forward_logits(const float *logits, const float *bias, int T, int N_r
                           int32_t *status, ebl_stream_t stream);
 
 /*
+ * router_forward_logits_balance -- router_forward_logits that also writes the
+ * per-tile statistics of the sequence-wise balance loss in the same pass over
+ * the logits (read from HBM once):
+ *   tile_psum[j, i] = sum over tokens t in [128 j, 128 j + 128), t < T, of
+ *                     s_{t,i} / sum_l s_{t,l}       (all N_r experts, no bias)
+ * next to tile_counts (required here); pair them with seq_balance_loss.
+ * Passage and reading as for router_forward_balance.  Indices, gates, counts
+ * and tile_counts are those of router_forward_logits, bit for bit.  The
+ * statistics use the fast fp32 score 1 / (1 + exp(-x)) (hardware exp2 and
+ * reciprocal approximations), not the rounded-once score that decides the
+ * selection: the loss is a training signal, not a selection, so one defined
+ * rounding is not needed there.  Each output is within 2^-16 relative (plus
+ * 2^-60 absolute) of the exact sums of the rounded-once scores for
+ * |x| <= 40; the sums run in a fixed order, so they are deterministic.  With
+ * N_r % 4 != 0 or a base address that is not 16-byte aligned, the routing
+ * runs in the row kernel and the statistics in a second pass that uses the
+ * fp64 score of balance_stats_logits (same tolerance or better).
+ * tile_counts  device, int32 [ceil(T/128), N_r], written, not NULL.
+ * tile_psum    device, fp32 [ceil(T/128), N_r], written, not NULL.
+ * Other arguments as router_forward_logits.
+ */
+int router_forward_logits_balance(const float *logits, const float *bias, int T, int N_r, int K,
+                                  int32_t *topk_idx, float *gates, int32_t *counts, int32_t *tile_counts,
+                                  float *tile_psum, int32_t *status, ebl_stream_t stream);
+
+/*
  * smebu_step -- one SMEBU update of the expert bias, once per optimizer step.
  * Passage: "SMEBU Load Balancing", "How it works", eqs. (23)-(28).
  *   nbar = sum_j n_j / N_r

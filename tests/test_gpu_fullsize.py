@@ -124,6 +124,19 @@ def test_logits_mode_full_tie_workload(cuda_device):
     assert np.all(np.abs(to_np(tp).astype(np.float64) - want) <= 2.0 ** -23 * want)
     r = oracle.seq_balance(scores, ref.idx, S, ebl.SEQ_BALANCE_ALPHA)
     assert np.allclose(to_np(loss_seq), r.loss_seq, rtol=1.2e-7, atol=0)
+    # the same statistics fused into the routing pass: routing bit for bit, the
+    # statistics within the fused tolerance (test_gpu_seq_balance)
+    from tests.test_gpu_seq_balance import FUSED_ATOL, FUSED_RTOL
+    c2 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc2 = torch.empty_like(tiles)
+    tp2 = torch.empty_like(tp)
+    idx2, gates2 = ebl.router_forward_logits_balance(x, bias, K, c2, tc2, tp2)
+    loss2, loss_seq2 = ebl.seq_balance_loss(tc2, tp2, T, K, S, ebl.SEQ_BALANCE_ALPHA)
+    torch.cuda.synchronize()
+    assert torch.equal(idx2, idx) and torch.equal(gates2, gates) and torch.equal(c2, counts)
+    assert torch.equal(tc2, tiles)
+    assert np.all(np.abs(to_np(tp2).astype(np.float64) - want) <= FUSED_RTOL * want + FUSED_ATOL)
+    assert np.allclose(to_np(loss_seq2), r.loss_seq, rtol=FUSED_RTOL, atol=0)
 
 
 def test_dispatch_combine_full_size(cuda_device):

@@ -19,6 +19,18 @@ into the per-sequence and batch values.  Tolerances:
     tile_psum entry is within one fp32 rounding (2^-24 relative, taken as
     2^-23 for the fp64 summation order) of the oracle, and the loss, a sum of
     positive terms each off by at most that much, within 1.2e-7 relative.
+  - Logits mode, statistics fused into the routing pass
+    (router_forward_logits_balance): the routing outputs are
+    router_forward_logits' bit for bit; the statistics use the fast fp32
+    score.  Its relative error is at most (1 - s)(2 + 1.173 |x|) ulp from the
+    fast exp, 0.5 ulp from 1 + e and 2 ulp from the fast reciprocal: 52 ulp
+    (6.2e-6) at |x| = 40 and 10 ulp (1.2e-6) at |x| <= 6.  The row total
+    (32 terms per lane, 3 shuffle adds) adds at most 35 ulp relative, 1/total
+    and the product 1.5 ulp, the fixed-order sum over the tile's rows (8 per
+    lane, 2 shuffle adds, 3 warp adds) 13 ulp: at most 2^-16 relative in
+    all (8.4e-6 at |x| = 40); scores below 2^-126 and above exp overflow are
+    covered by an absolute 2^-60.  The loss, a positive combination of the
+    entries, within 2^-16 relative too.
 """
 import numpy as np
 import pytest
@@ -33,6 +45,8 @@ pytestmark = pytest.mark.gpu
 
 PSUM_RTOL = 2e-5
 PSUM_ATOL = 1e-6 * 128
+FUSED_RTOL = 2.0 ** -16
+FUSED_ATOL = 2.0 ** -60
 
 # T, d, N_r, K, seq_len: ragged last tiles, both epilogue layouts (N_r % 64 == 0
 # splits the experts over two warp groups, else one), K from 1 to 8
@@ -205,3 +219,88 @@ def test_logits_mode_loss_end_to_end(cuda_device, T, Nr, K, S):
     r = oracle.seq_balance(ref.scores.astype(np.float64), ref.idx, S, alpha)
     assert np.allclose(to_np(loss_seq), r.loss_seq, rtol=1.2e-7, atol=0), (to_np(loss_seq), r.loss_seq)
     assert abs(float(loss.item()) - r.loss) <= 1.2e-7 * r.loss
+
+
+def _fused(xd, bias, K):
+    T, Nr = xd.shape
+    dev = xd.device
+    tiles = (T + 127) // 128
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.full((tiles, Nr), -1, dtype=torch.int32, device=dev)
+    tp = torch.full((tiles, Nr), -1.0, device=dev)
+    idx, g = ebl.router_forward_logits_balance(xd, bias, K, counts, tc, tp)
+    return idx, g, counts, tc, tp
+
+
+@pytest.mark.parametrize("misalign", [False, True])
+@pytest.mark.parametrize("T,Nr,K", LOGITS_CASES + [(3000, 256, 4), (1100, 128, 8)])
+def test_logits_mode_fused_balance(cuda_device, T, Nr, K, misalign):
+    """router_forward_logits_balance: routing identical to router_forward_logits
+    (and to the oracle), tile_psum within the fused tolerance of the oracle's
+    fp64 sums of the rounded-once scores.  misalign: the logits 4 bytes past a
+    16-byte boundary (the row kernel plus the separate statistics pass)."""
+    rng = np.random.default_rng(7 * T + Nr)
+    x = (rng.standard_normal((T, Nr)) * 3).astype(np.float32)
+    x[: T // 3] = np.round(x[: T // 3] * 8) / 8
+    x[T // 2, : min(Nr, 6)] = [88.7, -88.7, -103.0, -104.0, 700.0, -3e38][: min(Nr, 6)]
+    b = (rng.integers(-3, 4, Nr) * 0.01).astype(np.float32)
+    dev = cuda_device
+    if misalign:
+        buf = torch.empty(T * Nr + 1, device=dev)
+        buf[1:] = torch.from_numpy(x).reshape(-1).to(dev)
+        xd = buf[1:].view(T, Nr)
+    else:
+        xd = torch.from_numpy(x).to(dev)
+    bd = torch.from_numpy(b).to(dev)
+    idx, g, counts, tc, tp = _fused(xd, bd, K)
+    c2 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc2 = torch.empty_like(tc)
+    idx2, g2 = ebl.router_forward_logits(xd, bd, K, c2, tile_counts=tc2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(g, g2) and torch.equal(counts, c2) and torch.equal(tc, tc2)
+    ref = oracle.router_logits(x, b, K, want_scores=True, tile_tokens=128)
+    assert np.array_equal(to_np(idx), ref.idx) and np.array_equal(to_np(g), ref.gates)
+    assert np.array_equal(to_np(tc), ref.tile_counts)
+    want = oracle.tile_psum(ref.scores.astype(np.float64), 128)
+    got = to_np(tp).astype(np.float64)
+    err = np.abs(got - want)
+    assert np.all(err <= FUSED_RTOL * want + FUSED_ATOL), (err / np.maximum(want, 1e-300)).max()
+    rows = np.minimum(128, T - 128 * np.arange(want.shape[0]))
+    assert np.allclose(got.sum(1), rows, rtol=1e-5, atol=0)          # each row's normalised scores sum to 1
+    print("fused logits-mode tile_psum max rel err %.3e (tolerance %.3e)"
+          % ((err / np.maximum(want, 1e-30)).max(), FUSED_RTOL))
+
+
+@pytest.mark.parametrize("T,Nr,K,S", [(4096, 256, 4, 1024), (1536, 64, 8, 512), (2560, 128, 2, 256)])
+def test_logits_mode_fused_loss_end_to_end(cuda_device, T, Nr, K, S):
+    rng = np.random.default_rng(5 * T + Nr)
+    x = np.round(rng.standard_normal((T, Nr)).astype(np.float32) * 8) / 8
+    b = (rng.integers(-2, 3, Nr) * 0.01).astype(np.float32)
+    dev = cuda_device
+    idx, g, counts, tc, tp = _fused(torch.from_numpy(x).to(dev), torch.from_numpy(b).to(dev), K)
+    alpha = ebl.SEQ_BALANCE_ALPHA
+    loss, loss_seq = ebl.seq_balance_loss(tc, tp, T, K, S, alpha)
+    torch.cuda.synchronize()
+    ref = oracle.router_logits(x, b, K, want_scores=True, tile_tokens=128)
+    assert np.array_equal(to_np(tc), ref.tile_counts)
+    r = oracle.seq_balance(ref.scores.astype(np.float64), ref.idx, S, alpha)
+    assert np.allclose(to_np(loss_seq), r.loss_seq, rtol=FUSED_RTOL, atol=0), (to_np(loss_seq), r.loss_seq)
+    assert abs(float(loss.item()) - r.loss) <= FUSED_RTOL * r.loss
+
+
+def test_logits_mode_fused_balance_empty_and_checks(cuda_device):
+    dev = cuda_device
+    Nr = 64
+    x = torch.empty(0, Nr, device=dev)
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.empty(0, Nr, dtype=torch.int32, device=dev)
+    tp = torch.empty(0, Nr, device=dev)
+    idx, g = ebl.router_forward_logits_balance(x, torch.zeros(Nr, device=dev), 4, counts, tc, tp)
+    torch.cuda.synchronize()
+    assert idx.numel() == 0 and int(counts.sum().item()) == 0
+    rc = ebl.lib().router_forward_logits_balance(ebl._ptr(torch.zeros(256, Nr, device=dev)),
+                                                 ebl._ptr(torch.zeros(Nr, device=dev)), 256, Nr, 4,
+                                                 ebl._ptr(torch.zeros(256, 4, dtype=torch.int32, device=dev)),
+                                                 ebl._ptr(torch.zeros(256, 4, device=dev)), ebl._ptr(counts),
+                                                 None, ebl._ptr(torch.zeros(2, Nr, device=dev)), None, None)
+    assert rc == ebl.EBL_EINVAL                                         # tile_counts is required
