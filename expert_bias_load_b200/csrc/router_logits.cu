@@ -89,6 +89,21 @@ struct TopValues {
             }
         }
     }
+    // The Kth largest (1-based) of this lane's list and lane (lane ^ m)'s, both
+    // sorted descending, Kth <= P: taking i values from one list and Kth - i
+    // from the other, the Kth largest of the union is the largest over i of
+    // the smaller of the two lists' last values taken.  Both lanes get it.
+    template <int Kth>
+    __device__ __forceinline__ float kth_of_merge_xor(int m) const {
+        static_assert(Kth >= 1 && Kth <= K, "Kth within the list");
+        float o[Kth];
+#pragma unroll
+        for (int k = 0; k < Kth; ++k) o[k] = __shfl_xor_sync(0xffffffffu, v[k], m);
+        float r = fmaxf(v[Kth - 1], o[Kth - 1]);
+#pragma unroll
+        for (int i = 1; i < Kth; ++i) r = fmaxf(r, fminf(v[i - 1], o[Kth - 1 - i]));
+        return r;
+    }
 };
 
 // The warp's rows row0 .. row0+31 (lane l owns row0 + l): calls f(c, x) for
@@ -253,7 +268,12 @@ __device__ __forceinline__ float candidate_limit(float tau, float key_err = kKey
     return fmaxf(tau - (2.0f * key_err + 0x1p-19f * fabsf(tau)), -FLT_MAX);
 }
 
-constexpr int kStages = 2;  // row groups of a warp in the shared-memory ring: one loads while one is ranked
+// An unsigned value that orders like the float f (-inf lowest; f not NaN,
+// and +0 for zero, which every key here is: s >= +0 and +0 + -0 = +0).
+__device__ __forceinline__ uint32_t order_bits(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 __device__ __forceinline__ void cp_async_16(void *dst, const void *src, bool pred) {
     const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
@@ -266,10 +286,14 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// dynamic shared memory of the vector kernel: the logits ring
+// Dynamic shared memory of the vector kernel: one logits stage per warp (the
+// warp's 4 rows of the current item).  The stage is refilled as soon as each
+// candidate's logit has been copied out of it, and the candidate stage runs
+// while the next item loads; a single stage keeps 7 CTAs (28 warps) resident
+// per SM, which measured faster than two stages at 5 CTAs.
 template <int NV>
 constexpr size_t vec_ring_bytes() {
-    return sizeof(float) * kWarpsPerCta * kStages * kRowsPerGroup * 32 * NV;
+    return sizeof(float) * kWarpsPerCta * kRowsPerGroup * 32 * NV;
 }
 
 // Per-warp candidate buffers of the vector kernel.  With the balance option a
@@ -308,7 +332,6 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     extern __shared__ __align__(16) float ring_s[];  // [warp][stage][row of group][kRow]
     // tanh form: fl(0.5 + b); balance option: b.  -inf past N_r either way.
     __shared__ __align__(16) float hb_s[kMaxExperts];
-    __shared__ float bias_s[kMaxExperts];
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
     __shared__ __align__(16) WarpCand cand[kWarpsPerCta];
@@ -319,7 +342,6 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     for (int i = threadIdx.x; i < kMaxExperts; i += kThreads) {
         const bool in = i < Nr;
         const float b = in ? bias[i] : 0.0f;
-        bias_s[i] = b;
         hb_s[i] = in ? (BAL ? b : __fadd_rn(0.5f, b)) : -INFINITY;
         hist_total[i] = 0;
         hist_tile[i] = 0;
@@ -338,7 +360,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     const int lane = threadIdx.x & 31;
     const int r = lane >> 3;  // row of the group this lane works on
     const int j = lane & 7;   // lane within the row: float4 columns j, j + 8, j + 16, ...
-    float *ring = ring_s + (size_t)warp * kStages * kRowsPerGroup * kRow;
+    float *ring = ring_s + (size_t)warp * kRowsPerGroup * kRow;
     int *cc = cand[warp].c[r];
     float *ck = cand[warp].key[r];
     float *cs = cand[warp].s[r];
@@ -348,7 +370,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     int *sc = sel_c[warp][r];
 
     // Work item i of this warp: row group i % 8 of tile blockIdx.x + (i / 8) * gridDim.x.
-    // Its 4 rows go to ring stage i % kStages; lane j of a row copies float4
+    // Its 4 rows go to the warp's stage; lane j of a row copies float4
     // columns 8m + j, so each copy instruction covers 128 contiguous bytes of
     // each of the 4 rows.  Rows past T are zero-filled without a read.  (Whole
     // tiles per CTA also stream 128 KB of consecutive rows at a time, which
@@ -360,7 +382,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     auto issue = [&](int item, int64_t row) {
         const bool rin = row < T;
         const float *src = logits + (rin ? row : 0) * (int64_t)Nr;
-        float *dst = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;
+        float *dst = ring + r * kRow;
 #pragma unroll
         for (int m = 0; m < NV; ++m) {
             const int c = 4 * (8 * m + j);
@@ -376,7 +398,6 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     const int items = num_tiles > (int)blockIdx.x
                           ? ((num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * kGroupsPerWarp
                           : 0;
-    static_assert(kStages == 2, "one item in flight while one is ranked");
     float psum[BAL ? NV : 1][4];  // balance option: this lane's column sums over the tile's rows it sees
 #pragma unroll
     for (int m = 0; m < (BAL ? NV : 1); ++m)
@@ -387,10 +408,9 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     for (int item = 0; item < items; ++item) {
         const int64_t row = ahead;
         ahead = next_row(ahead, item);
-        issue(item + 1, ahead);  // into the stage the previous item released
-        cp_async_wait<kStages - 1>();
+        cp_async_wait<0>();
         __syncwarp();
-        const float *xr = ring + ((item % kStages) * kRowsPerGroup + r) * kRow;  // this lane's row
+        const float *xr = ring + r * kRow;  // this lane's row; the next item is issued once it is read
 
         // approximate keys of this lane's 4*NV experts
         float kv[NV][4];
@@ -473,8 +493,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         }
         top.merge_xor(1);
         top.merge_xor(2);
-        top.merge_xor(4);
-        const float lim = candidate_limit(top.v[K - 1], kErr);
+        const float lim = candidate_limit(top.template kth_of_merge_xor<K>(4), kErr);
         unsigned mask = 0;
 #pragma unroll
         for (int m = 0; m < NV; ++m)
@@ -503,28 +522,31 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
             for (int q = 0; q < 4; ++q) {
                 const int p = __ffs(mm) - 1;
                 mm &= mm - 1;
-                if (q < n) cc[excl + q] = 4 * (8 * (p >> 2) + j) + (p & 3);
+                const int col = 4 * (8 * (p >> 2) + j) + (p & 3);
+                if (q < n) {
+                    cc[excl + q] = col;
+                    ck[excl + q] = xr[col];
+                }
             }
             __syncwarp();
+            issue(item + 1, ahead);  // every candidate's logit is in ck: the stage is free
             const bool has = j < row_n;
             int c = has ? cc[j] : 0;
-            const float s = sigmoid_rounded_once(xr[c]);
-            const float key = has ? __fadd_rn(s, bias_s[c]) : -INFINITY;
-            c = has ? c : 0x7fffffff;
+            const float s = sigmoid_rounded_once(ck[has ? j : 0]);
+            const uint64_t ord =
+                has ? ((uint64_t)order_bits(__fadd_rn(s, __ldg(bias + c))) << 32) | (uint32_t)~c : 0ull;
             int rank = 0;
 #pragma unroll
-            for (int d = 1; d < kLanesPerRow; ++d) {
-                const int src = (lane & ~(kLanesPerRow - 1)) | ((j + d) & (kLanesPerRow - 1));
-                const float ko = __shfl_sync(0xffffffffu, key, src);
-                const int co = __shfl_sync(0xffffffffu, c, src);
-                rank += (ko > key || (ko == key && co < c)) ? 1 : 0;
-            }
+            for (int d = 1; d < kLanesPerRow; ++d)
+                rank += __shfl_sync(0xffffffffu, ord, (lane & ~(kLanesPerRow - 1)) | ((j + d) & (kLanesPerRow - 1))) > ord
+                            ? 1 : 0;
             if (has && rank < K) {
                 ss[rank] = s;
                 sc[rank] = c;
             }
             __syncwarp();
         } else {
+            issue(item + 1, ahead);  // this path reads the candidates' logits from global memory (L2)
             const int most = __reduce_max_sync(0xffffffffu, row_n);
             // rounds of up to kWin candidates per row (one round unless many keys tie)
             for (int w0 = 0; w0 < most; w0 += kWin) {
@@ -544,9 +566,9 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                 // slots [wn, 8) get a sentinel that ranks below everything
                 for (int e = j; e < wn; e += kLanesPerRow) {
                     const int c = cc[e];
-                    const float s = sigmoid_rounded_once(xr[c]);
+                    const float s = sigmoid_rounded_once(__ldg(logits + row * (int64_t)Nr + c));
                     cs[e] = s;
-                    ck[e] = __fadd_rn(s, bias_s[c]);
+                    ck[e] = __fadd_rn(s, __ldg(bias + c));
                 }
                 if (j >= wn) {
                     ck[j] = -INFINITY;
