@@ -20,8 +20,10 @@
 // usual case) gives each token row to 8 lanes: every load instruction fetches
 // 128 contiguous bytes of each of 4 rows, a lane's 4*NV logits and their keys
 // stay in registers, tau comes from a butterfly over the 8 lanes, and the
-// candidates are compacted per row in shared memory, scored by the row's 8
-// lanes and ranked in parallel.  The logits are read from HBM exactly once.
+// candidates (column and logit) are compacted per row in shared memory, scored
+// by the row's 8 lanes and ranked in parallel while the next rows load.  The
+// logits are read from HBM exactly once.  With the balance option the same
+// pass also writes the per-tile statistics of the sequence-wise balance loss.
 // The row kernel (any N_r, 4-byte alignment) gives each row to one thread and
 // reads the logits twice.
 
@@ -296,7 +298,8 @@ constexpr size_t vec_ring_bytes() {
     return sizeof(float) * kWarpsPerCta * kRowsPerGroup * 32 * NV;
 }
 
-// Per-warp candidate buffers of the vector kernel.  With the balance option a
+// Per-warp candidate buffers of the vector kernel (the fast path lists each
+// candidate's column in c and its logit in key).  With the balance option a
 // warp's column sums (kMaxExperts floats) reuse this space at the end of each
 // tile, after the warp's last candidate stage of the tile.
 struct WarpCand {
