@@ -2,7 +2,8 @@
 logits mode bit-exact (both kernels: aligned and misaligned logits), GEMM mode
 under the near-tie rule, dispatch and combine bit-exact, the bias updates
 (SMEBU clamped and linear over several layers, the sign update), and the
-sequence-wise balance statistics.  Each case
+sequence-wise balance statistics (GEMM mode, and logits mode fused into the
+routing pass).  Each case
 draws its sizes, the bias pattern and the value distribution from its own seed."""
 import numpy as np
 import pytest
@@ -192,3 +193,45 @@ def test_balance_option_random_shapes(cuda_device, case):
     r = oracle.seq_balance(ref.scores, ref.idx, S, alpha)
     excused = (ref.gap < 1e-3).reshape(T // S, S).sum(1)
     assert np.all(np.abs(to_np(loss_seq) - r.loss_seq) <= 2e-5 * r.loss_seq + excused * alpha * Nr / S)
+
+
+@pytest.mark.parametrize("case", list(range(12)))
+def test_logits_mode_fused_balance_random_shapes(cuda_device, case):
+    """router_forward_logits_balance on seeded random shapes: routing bit for
+    bit that of router_forward_logits and the oracle's, the per-tile statistics
+    within the fused tolerance (2^-16 relative + 2^-60) of the oracle's fp64
+    sums of the rounded-once scores."""
+    rng = np.random.default_rng(3000 + case)
+    T = int(rng.integers(1, 3000))
+    Nr = int(rng.choice([int(rng.integers(1, 257)), 4 * int(rng.integers(1, 65))]))
+    K = int(rng.integers(1, min(8, Nr) + 1))
+    scale = float(rng.choice([1.0, 4.0, 0.125]))
+    x = (rng.standard_normal((T, Nr)) * scale).astype(np.float32)
+    if rng.integers(0, 2):
+        x = np.round(x * 8) / 8
+    b = _bias(rng, Nr)
+    dev = cuda_device
+    misalign = bool(rng.integers(0, 2))
+    if misalign:
+        buf = torch.empty(T * Nr + 1, dtype=torch.float32, device=dev)
+        buf[1:] = torch.from_numpy(x.reshape(-1)).to(dev)
+        xd = buf[1:].view(T, Nr)
+    else:
+        xd = torch.from_numpy(x).to(dev)
+    bd = torch.from_numpy(b).to(dev)
+    tiles_n = (T + 127) // 128
+    counts = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc = torch.full((tiles_n, Nr), -1, dtype=torch.int32, device=dev)
+    tp = torch.full((tiles_n, Nr), -1.0, device=dev)
+    idx, g = ebl.router_forward_logits_balance(xd, bd, K, counts, tc, tp)
+    c2 = torch.zeros(Nr, dtype=torch.int32, device=dev)
+    tc2 = torch.empty_like(tc)
+    idx2, g2 = ebl.router_forward_logits(xd, bd, K, c2, tile_counts=tc2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(g, g2) and torch.equal(counts, c2) and torch.equal(tc, tc2)
+    ref = oracle.router_logits(x, b, K, tile_tokens=128, want_scores=True)
+    assert np.array_equal(to_np(idx), ref.idx), (T, Nr, K, misalign)
+    assert np.array_equal(to_np(tc), ref.tile_counts)
+    want = oracle.tile_psum(ref.scores.astype(np.float64), 128)
+    got = to_np(tp).astype(np.float64)
+    assert np.all(np.abs(got - want) <= 2.0 ** -16 * want + 2.0 ** -60), (T, Nr, K, misalign)
