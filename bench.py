@@ -253,6 +253,21 @@ def suite_cpu(seconds, threads_label):
         t = run(rows, 2)
         out.append({"workload": name, "mode": mode, "rows": rows, "seconds": t, "tokens_per_s": rows / t,
                     "extrapolated": rows < T})
+    if threads_label == "one_thread":
+        # the bias updates alone, per step, at N_r = 256 on loads of the tie workload's size
+        counts = np.bincount(np.random.default_rng(5).integers(0, 256, 4 * 1048576), minlength=256).astype(np.int64)
+        b = synth.dead_start_bias(256).numpy()
+        m = np.zeros(256, np.float32)
+        reps = 2000
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.smebu(counts, b, m)
+        t_smebu = (time.perf_counter() - t0) / reps
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.sign_update(counts, b)
+        t_sign = (time.perf_counter() - t0) / reps
+        out.append({"workload": "ties", "mode": "updates", "smebu_us": t_smebu * 1e6, "sign_us": t_sign * 1e6})
     return out
 
 
@@ -285,6 +300,20 @@ def cpu_baseline_suite(seconds, dev):
         return ev[0].elapsed_time(ev[1]) / reps
 
     entries = []
+    # the bias updates alone: one CTA per step, 1000 back-to-back launches per CUDA-event pair
+    counts = torch.bincount(torch.randint(0, 256, (4 * 1048576,), generator=torch.Generator().manual_seed(5)),
+                            minlength=256).to(torch.int32).to(dev)
+    b = synth.dead_start_bias(256, device=dev)
+    m = torch.zeros(256, device=dev)
+    upd = {"workload": "ties", "step": "bias update alone (N_r = 256), per step",
+           "gpu_smebu_us": gpu_ms(lambda: ebl.smebu_step(counts, b, m), reps=1000) * 1e3,
+           "gpu_sign_us": gpu_ms(lambda: ebl.sign_update_step(counts, b, 1e-3), reps=1000) * 1e3,
+           "note": "GPU: per launch from Python, which the host's launch rate bounds; oracle: one thread, "
+                   "per call through ctypes"}
+    for r in cpu["one_thread"][1]:
+        if r.get("mode") == "updates":
+            upd["oracle_smebu_us"] = r["smebu_us"]
+            upd["oracle_sign_us"] = r["sign_us"]
     for name, mode, _, _ in SUITE_ENTRIES:
         c = synth.WORKLOADS[name]
         T, d, Nr, K = c["T"], c["d"], c["Nr"], c["K"]
@@ -337,6 +366,7 @@ def cpu_baseline_suite(seconds, dev):
         entries.append(e)
         del fn
         torch.cuda.empty_cache()
+    entries.append(upd)
     return {"entries": entries, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
             "note": "oracle samples sized for about %.0f s each; a sample smaller than T is extrapolated "
                     "linearly; GPU inputs resident" % seconds}

@@ -37,6 +37,9 @@ def test_oracle_suite_child_lines():
                            timeout=600)
         assert r.returncode == 0, r.stderr[-2000:]
         res = json.loads(r.stdout.strip().splitlines()[-1])
+        if mode == 1:                                   # the one-thread child also times the bias updates alone
+            upd = res.pop()
+            assert upd["mode"] == "updates" and upd["smebu_us"] > 0 and upd["sign_us"] > 0
         assert [(e["workload"], e["mode"]) for e in res] == entries
         for e in res:
             assert e["rows"] >= 1 and e["seconds"] > 0 and e["tokens_per_s"] > 0
