@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     static_assert(NV % 2 == 0 && kRow <= kMaxExperts, "a lane holds NV float4 of a row, in pairs");
     // distance of the approximate key to the exact one (see key_approx, sigmoid_fast)
     constexpr float kErr = BAL ? kSigmaErr : kKeyErr;
-    extern __shared__ __align__(16) float ring_s[];  // [warp][stage][row of group][kRow]
+    extern __shared__ __align__(16) float ring_s[];  // [warp][row of group][kRow]
     // tanh form: fl(0.5 + b); balance option: b.  -inf past N_r either way.
     __shared__ __align__(16) float hb_s[kMaxExperts];
     __shared__ int hist_total[kMaxExperts];
