@@ -232,8 +232,12 @@ def _fused(xd, bias, K):
     return idx, g, counts, tc, tp
 
 
+# vector-kernel shapes with padding columns (N_r % 4 == 0 but below the lanes' column blocks)
+FUSED_EXTRA = [(3000, 256, 4), (1100, 128, 8), (777, 4, 2), (500, 68, 6), (500, 132, 3), (600, 252, 8)]
+
+
 @pytest.mark.parametrize("misalign", [False, True])
-@pytest.mark.parametrize("T,Nr,K", LOGITS_CASES + [(3000, 256, 4), (1100, 128, 8)])
+@pytest.mark.parametrize("T,Nr,K", LOGITS_CASES + FUSED_EXTRA)
 def test_logits_mode_fused_balance(cuda_device, T, Nr, K, misalign):
     """router_forward_logits_balance: routing identical to router_forward_logits
     (and to the oracle), tile_psum within the fused tolerance of the oracle's
