@@ -235,12 +235,19 @@ __global__ void __launch_bounds__(kThreads) router_logits_kernel(const float *__
 constexpr int kLanesPerRow = 8;
 constexpr int kRowsPerGroup = 32 / kLanesPerRow;         // rows a warp takes at once
 constexpr int kGroupsPerWarp = 32 / kRowsPerGroup;       // row groups of a warp per tile
-constexpr int kWin = 32;                                 // candidates of a row scored per round
+constexpr int kWin = 24;                                 // candidates of a row scored per round
 constexpr int kWinPad = kWin + 1;                        // odd stride: rows of a group hit different banks
 
 __device__ __forceinline__ float tanh_approx(float x) {
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// The largest of three values; NaN inputs are ignored like fmaxf does.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
 
@@ -288,6 +295,21 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// Lane j of a row owns the row's 4*NV consecutive columns [4*NV*j, 4*NV*(j+1)),
+// so the row's candidates come out of a prefix over its lanes already in
+// expert order.  In shared memory (the logits stage and the bias table) each
+// lane's columns are followed by 16 unused bytes: a lane reads its float4 m at
+// 16 (NV + 1) j + 16 m bytes, and NV + 1 odd puts the 8 lanes of a row on 8
+// different 16-byte bank groups.  Column c sits at float offset pad_col(c).
+template <int NV>
+__device__ __forceinline__ int pad_col(int c) {
+    return c + 4 * (c / (4 * NV));
+}
+template <int NV>
+__host__ __device__ constexpr int padded_row() {
+    return 32 * (NV + 1);  // floats of one row (or the bias table) in shared memory
+}
+
 // Dynamic shared memory of the vector kernel: one logits stage per warp (the
 // warp's 4 rows of the current item).  The stage is refilled as soon as each
 // candidate's logit has been copied out of it, and the candidate stage runs
@@ -295,7 +317,7 @@ __device__ __forceinline__ void cp_async_wait() {
 // per SM, which measured faster than two stages at 5 CTAs.
 template <int NV>
 constexpr size_t vec_ring_bytes() {
-    return sizeof(float) * kWarpsPerCta * kRowsPerGroup * 32 * NV;
+    return sizeof(float) * kWarpsPerCta * kRowsPerGroup * padded_row<NV>();
 }
 
 // Per-warp candidate buffers of the vector kernel (the fast path lists each
@@ -307,7 +329,7 @@ struct WarpCand {
     float key[kRowsPerGroup][kWinPad];
     float s[kRowsPerGroup][kWinPad];
 };
-static_assert(sizeof(WarpCand) >= kMaxExperts * sizeof(float), "column sums fit the candidate buffers");
+static_assert(sizeof(WarpCand) >= (kMaxExperts + 32) * sizeof(float), "column sums fit the candidate buffers");
 
 // BAL (the balance option): the approximate key is sigmoid_fast(x) + b instead
 // of the tanh form, and the same fast scores give the per-tile statistics of
@@ -317,24 +339,24 @@ static_assert(sizeof(WarpCand) >= kMaxExperts * sizeof(float), "column sums fit 
 // lanes per column with two shuffles and the CTA adds its four warps in
 // order, so the sums do not depend on scheduling.
 template <int K, int NV, bool FULL, bool BAL>
-__global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float *__restrict__ logits,
-                                                                     const float *__restrict__ bias, int T, int Nr,
-                                                                     int32_t *__restrict__ topk_idx,
-                                                                     float *__restrict__ gates,
-                                                                     int32_t *__restrict__ counts,
-                                                                     int32_t *__restrict__ tile_counts,
-                                                                     float *__restrict__ tile_psum,
-                                                                     int32_t *__restrict__ status) {
+__device__ __forceinline__ void logits_vec_body(const float *__restrict__ logits, const float *__restrict__ bias,
+                                                int T, int Nr, int32_t *__restrict__ topk_idx,
+                                                float *__restrict__ gates, int32_t *__restrict__ counts,
+                                                int32_t *__restrict__ tile_counts, float *__restrict__ tile_psum,
+                                                int32_t *__restrict__ status) {
     // lane-local lists of the approximate pass hold P >= K values (P a power of two)
     constexpr int P = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
-    constexpr int kRow = 32 * NV;  // floats per row in the ring (N_r rounded up, zero-filled)
+    constexpr int kRow = 32 * NV;  // columns per row in the ring (N_r rounded up, zero-filled)
+    constexpr int kRowPad = padded_row<NV>();
+    constexpr int kLaneCols = 4 * NV;  // columns a lane owns
     // FULL: N_r == kRow, so every column a lane copies exists (no per-column test)
     static_assert(NV % 2 == 0 && kRow <= kMaxExperts, "a lane holds NV float4 of a row, in pairs");
     // distance of the approximate key to the exact one (see key_approx, sigmoid_fast)
     constexpr float kErr = BAL ? kSigmaErr : kKeyErr;
-    extern __shared__ __align__(16) float ring_s[];  // [warp][row of group][kRow]
+    extern __shared__ __align__(16) float ring_s[];  // [warp][row of group][kRowPad]
     // tanh form: fl(0.5 + b); balance option: b.  -inf past N_r either way.
-    __shared__ __align__(16) float hb_s[kMaxExperts];
+    // Padded like a row of the ring.
+    __shared__ __align__(16) float hb_s[kMaxExperts + 32];
     __shared__ int hist_total[kMaxExperts];
     __shared__ int hist_tile[kMaxExperts];
     __shared__ __align__(16) WarpCand cand[kWarpsPerCta];
@@ -343,11 +365,13 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     __shared__ int sel_c[kWarpsPerCta][kRowsPerGroup][2 * K];
 
     for (int i = threadIdx.x; i < kMaxExperts; i += kThreads) {
-        const bool in = i < Nr;
-        const float b = in ? bias[i] : 0.0f;
-        hb_s[i] = in ? (BAL ? b : __fadd_rn(0.5f, b)) : -INFINITY;
         hist_total[i] = 0;
         hist_tile[i] = 0;
+    }
+    for (int i = threadIdx.x; i < kRow; i += kThreads) {
+        const bool in = i < Nr;
+        const float b = in ? bias[i] : 0.0f;
+        hb_s[pad_col<NV>(i)] = in ? (BAL ? b : __fadd_rn(0.5f, b)) : -INFINITY;
     }
     for (int i = threadIdx.x; i < kWarpsPerCta * kRowsPerGroup * 2 * K; i += kThreads) {
         (&sel_key[0][0][0])[i] = -INFINITY;
@@ -362,8 +386,9 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int r = lane >> 3;  // row of the group this lane works on
-    const int j = lane & 7;   // lane within the row: float4 columns j, j + 8, j + 16, ...
-    float *ring = ring_s + (size_t)warp * kRowsPerGroup * kRow;
+    const int j = lane & 7;   // lane within the row: it owns columns [4*NV*j, 4*NV*(j+1))
+    float *ring = ring_s + (size_t)warp * kRowsPerGroup * kRowPad;
+    const float *hbl = hb_s + (kLaneCols + 4) * j;  // this lane's bias values
     int *cc = cand[warp].c[r];
     float *ck = cand[warp].key[r];
     float *cs = cand[warp].s[r];
@@ -374,8 +399,9 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
 
     // Work item i of this warp: row group i % 8 of tile blockIdx.x + (i / 8) * gridDim.x.
     // Its 4 rows go to the warp's stage; lane j of a row copies float4
-    // columns 8m + j, so each copy instruction covers 128 contiguous bytes of
-    // each of the 4 rows.  Rows past T are zero-filled without a read.  (Whole
+    // columns 8m + j (into the owner lane's padded slots), so each copy
+    // instruction covers 128 contiguous bytes of each of the 4 rows.  Rows
+    // past T are zero-filled without a read.  (Whole
     // tiles per CTA also stream 128 KB of consecutive rows at a time, which
     // measured 2% faster than dealing row groups to all warps in turn.)
     auto item_row = [&](int item) -> int64_t {
@@ -385,12 +411,12 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     auto issue = [&](int item, int64_t row) {
         const bool rin = row < T;
         const float *src = logits + (rin ? row : 0) * (int64_t)Nr;
-        float *dst = ring + r * kRow;
+        float *dst = ring + r * kRowPad;
 #pragma unroll
         for (int m = 0; m < NV; ++m) {
             const int c = 4 * (8 * m + j);
             const bool ok = FULL ? rin : (rin && c < Nr);
-            cp_async_16(dst + c, src + (ok ? c : 0), ok);
+            cp_async_16(dst + pad_col<NV>(c), src + (ok ? c : 0), ok);
         }
         cp_async_commit();
     };
@@ -413,7 +439,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         ahead = next_row(ahead, item);
         cp_async_wait<0>();
         __syncwarp();
-        const float *xr = ring + r * kRow;  // this lane's row; the next item is issued once it is read
+        // this lane's columns of its row; the next item is issued once they are read
+        const float *xr = ring + r * kRowPad + (kLaneCols + 4) * j;
 
         // approximate keys of this lane's 4*NV experts
         float kv[NV][4];
@@ -423,7 +450,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
             float rs = 0.0f;
 #pragma unroll
             for (int m = 0; m < NV; ++m) {
-                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
+                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * m);
                 kv[m][0] = sigmoid_fast(x.x);
                 kv[m][1] = sigmoid_fast(x.y);
                 kv[m][2] = sigmoid_fast(x.z);
@@ -431,7 +458,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if constexpr (!FULL)  // padding columns (zero-filled, s = 1/2) add nothing
-                        if (4 * (8 * m + j) + e >= Nr) kv[m][e] = 0.0f;
+                        if (kLaneCols * j + 4 * m + e >= Nr) kv[m][e] = 0.0f;
                     rs += kv[m][e];
                 }
             }
@@ -441,7 +468,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
             const float inv = (row < T && rs > 0.0f) ? __frcp_rn(rs) : 0.0f;
 #pragma unroll
             for (int m = 0; m < NV; ++m) {
-                const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
+                const float4 h = *reinterpret_cast<const float4 *>(hbl + 4 * m);
                 const float hv[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -452,8 +479,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         } else {
 #pragma unroll
             for (int m = 0; m < NV; ++m) {
-                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * (8 * m + j));
-                const float4 h = *reinterpret_cast<const float4 *>(&hb_s[4 * (8 * m + j)]);
+                const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * m);
+                const float4 h = *reinterpret_cast<const float4 *>(hbl + 4 * m);
                 kv[m][0] = key_approx(x.x, h.x);
                 kv[m][1] = key_approx(x.y, h.y);
                 kv[m][2] = key_approx(x.z, h.z);
@@ -466,9 +493,9 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         float gm[G];
 #pragma unroll
         for (int q = 0; q < G; ++q) {
-            const float a = fmaxf(fmaxf(kv[2 * q][0], kv[2 * q][1]), fmaxf(kv[2 * q][2], kv[2 * q][3]));
-            const float b = fmaxf(fmaxf(kv[2 * q + 1][0], kv[2 * q + 1][1]), fmaxf(kv[2 * q + 1][2], kv[2 * q + 1][3]));
-            gm[q] = fmaxf(a, b);
+            const float a = fmax3(kv[2 * q][0], kv[2 * q][1], kv[2 * q][2]);
+            const float b = fmax3(kv[2 * q][3], kv[2 * q + 1][0], kv[2 * q + 1][1]);
+            gm[q] = fmaxf(b, fmax3(kv[2 * q + 1][2], kv[2 * q + 1][3], a));
         }
         TopValues<P> top;
         top.init();
@@ -521,33 +548,77 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
         const int excl = incl - n;
         const int row_n = __shfl_sync(0xffffffffu, incl, lane | (kLanesPerRow - 1));
 
-        if (__all_sync(0xffffffffu, n <= 4 && row_n <= kLanesPerRow)) {
-            // The usual case, without loops: at most 4 candidates per lane and
-            // 8 per row.  Lane j scores the row's j-th candidate and ranks it
-            // against the other 7 through shuffles.
+        if (__all_sync(0xffffffffu, n <= 8 && row_n <= 2 * kLanesPerRow)) {
+            // The usual case, without loops: at most 8 candidates per lane and
+            // 16 per row (at most 4 and 8 on most items).  Lane j scores the
+            // row's j-th candidate (and its (j+8)-th, if any) and ranks it
+            // against the others through shuffles.
             unsigned mm = mask;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int p = __ffs(mm) - 1;
                 mm &= mm - 1;
-                const int col = 4 * (8 * (p >> 2) + j) + (p & 3);
                 if (q < n) {
-                    cc[excl + q] = col;
-                    ck[excl + q] = xr[col];
+                    cc[excl + q] = kLaneCols * j + p;
+                    ck[excl + q] = xr[p];
+                }
+            }
+            if (__any_sync(0xffffffffu, n > 4)) {
+#pragma unroll
+                for (int q = 4; q < 8; ++q) {
+                    const int p = __ffs(mm) - 1;
+                    mm &= mm - 1;
+                    if (q < n) {
+                        cc[excl + q] = kLaneCols * j + p;
+                        ck[excl + q] = xr[p];
+                    }
                 }
             }
             __syncwarp();
             issue(item + 1, ahead);  // every candidate's logit is in ck: the stage is free
             const bool has = j < row_n;
-            int c = has ? cc[j] : 0;
+            const int c = has ? cc[j] : 0;
             const float s = sigmoid_rounded_once(ck[has ? j : 0]);
-            const uint64_t ord =
-                has ? ((uint64_t)order_bits(__fadd_rn(s, __ldg(bias + c))) << 32) | (uint32_t)~c : 0ull;
+            // The row's list is in expert order, so an equal key ranks above
+            // exactly when it sits earlier in the list: lane q < j counts on
+            // o_q >= o, i.e. o_q > o - 1.  Keys order as o >= 0x007fffff (-inf);
+            // lanes past the list carry 0 and rank below everything.
+            const uint32_t o = has ? order_bits(__fadd_rn(s, __ldg(bias + c))) : 0u;
+            const int src0 = lane & ~(kLanesPerRow - 1);
             int rank = 0;
+            if (!__any_sync(0xffffffffu, row_n > kLanesPerRow)) {
 #pragma unroll
-            for (int d = 1; d < kLanesPerRow; ++d)
-                rank += __shfl_sync(0xffffffffu, ord, (lane & ~(kLanesPerRow - 1)) | ((j + d) & (kLanesPerRow - 1))) > ord
-                            ? 1 : 0;
+                for (int d = 1; d < kLanesPerRow; ++d) {
+                    const uint32_t oq = __shfl_sync(0xffffffffu, o, src0 | ((j + d) & (kLanesPerRow - 1)));
+                    // (two spellings of one test: each keeps its variant's register count lower)
+                    if constexpr (BAL)
+                        rank += (oq > o) | ((oq == o) & (j + d >= kLanesPerRow));
+                    else
+                        rank += oq > (o - (uint32_t)((j + d) >> 3)) ? 1 : 0;
+                }
+            } else {
+                // a second candidate per lane at list position j + 8, after
+                // every first one
+                const bool has2 = j + kLanesPerRow < row_n;
+                const int c2 = has2 ? cc[j + kLanesPerRow] : 0;
+                const float s2 = sigmoid_rounded_once(ck[has2 ? j + kLanesPerRow : 0]);
+                const uint32_t o2 = has2 ? order_bits(__fadd_rn(s2, __ldg(bias + c2))) : 0u;
+                rank = o2 > o ? 1 : 0;
+                int rank2 = o >= o2 ? 1 : 0;
+#pragma unroll
+                for (int d = 1; d < kLanesPerRow; ++d) {
+                    const int q = src0 | ((j + d) & (kLanesPerRow - 1));
+                    const uint32_t oq = __shfl_sync(0xffffffffu, o, q);
+                    const uint32_t oq2 = __shfl_sync(0xffffffffu, o2, q);
+                    const uint32_t before = (uint32_t)((j + d) >> 3);  // lane q precedes lane j
+                    rank += (oq > o - before ? 1 : 0) + (oq2 > o ? 1 : 0);
+                    rank2 += (oq >= o2 ? 1 : 0) + (oq2 > o2 - before ? 1 : 0);
+                }
+                if (has2 && rank2 < K) {
+                    ss[rank2] = s2;
+                    sc[rank2] = c2;
+                }
+            }
             if (has && rank < K) {
                 ss[rank] = s;
                 sc[rank] = c;
@@ -564,7 +635,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                     while (mm) {
                         const int p = __ffs(mm) - 1;
                         mm &= mm - 1;
-                        if (off >= w0 && off < w0 + kWin) cc[off - w0] = 4 * (8 * (p >> 2) + j) + (p & 3);
+                        if (off >= w0 && off < w0 + kWin) cc[off - w0] = kLaneCols * j + p;
                         ++off;
                     }
                 }
@@ -666,7 +737,7 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                         float v = psum[m][e];
                         v += __shfl_xor_sync(0xffffffffu, v, 8);
                         v += __shfl_xor_sync(0xffffffffu, v, 16);
-                        if (r == 0) colsum[4 * (8 * m + j) + e] = v;
+                        if (r == 0) colsum[(kLaneCols + 4) * j + 4 * m + e] = v;  // padded like hb_s
                         psum[m][e] = 0.0f;
                     }
             }
@@ -681,7 +752,8 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
                     const float *c1 = reinterpret_cast<const float *>(&cand[1]);
                     const float *c2 = reinterpret_cast<const float *>(&cand[2]);
                     const float *c3 = reinterpret_cast<const float *>(&cand[3]);
-                    tile_psum[(size_t)tile * Nr + e] = ((c0[e] + c1[e]) + c2[e]) + c3[e];
+                    const int pe = pad_col<NV>(e);
+                    tile_psum[(size_t)tile * Nr + e] = ((c0[pe] + c1[pe]) + c2[pe]) + c3[pe];
                 }
             }
             __syncthreads();
@@ -691,6 +763,29 @@ __global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float
     __syncthreads();
     for (int e = threadIdx.x; e < Nr; e += kThreads)
         if (hist_total[e] != 0) atomicAdd(&counts[e], hist_total[e]);
+}
+
+// Routing alone: the compiler's own register choice (64 at K = 4, N_r = 256)
+// gives 8 CTAs per SM.
+template <int K, int NV, bool FULL>
+__global__ void __launch_bounds__(kThreads) router_logits_vec_kernel(const float *__restrict__ logits,
+                                                                     const float *__restrict__ bias, int T, int Nr,
+                                                                     int32_t *__restrict__ topk_idx,
+                                                                     float *__restrict__ gates,
+                                                                     int32_t *__restrict__ counts,
+                                                                     int32_t *__restrict__ tile_counts,
+                                                                     int32_t *__restrict__ status) {
+    logits_vec_body<K, NV, FULL, false>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, nullptr, status);
+}
+
+// With the balance statistics: the lane's column sums hold 4*NV more
+// registers; 96 per thread keep 5 CTAs per SM.
+template <int K, int NV, bool FULL>
+__global__ void __launch_bounds__(kThreads, 5) router_logits_vec_balance_kernel(
+    const float *__restrict__ logits, const float *__restrict__ bias, int T, int Nr, int32_t *__restrict__ topk_idx,
+    float *__restrict__ gates, int32_t *__restrict__ counts, int32_t *__restrict__ tile_counts,
+    float *__restrict__ tile_psum, int32_t *__restrict__ status) {
+    logits_vec_body<K, NV, FULL, true>(logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, tile_psum, status);
 }
 
 // max over i of |approximate score - exact score| as the bits of a
@@ -746,7 +841,8 @@ template <int K, int NV, bool FULL, bool BAL>
 cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, int32_t *topk_idx, float *gates,
                        int32_t *counts, int32_t *tile_counts, float *tile_psum, int32_t *status, int num_sms,
                        cudaStream_t stream) {
-    const void *kern = reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL, BAL>);
+    const void *kern = BAL ? reinterpret_cast<const void *>(&router_logits_vec_balance_kernel<K, NV, FULL>)
+                           : reinterpret_cast<const void *>(&router_logits_vec_kernel<K, NV, FULL>);
     const size_t smem = vec_ring_bytes<NV>();
     int per_sm = 1;
     cudaError_t err = vec_setup(kern, smem, &per_sm);
@@ -754,9 +850,12 @@ cudaError_t launch_vec(const float *logits, const float *bias, int T, int Nr, in
     const int num_tiles = (T + kTileTokens - 1) / kTileTokens;
     int grid = num_sms * per_sm;
     if (grid > num_tiles) grid = num_tiles;
-    router_logits_vec_kernel<K, NV, FULL, BAL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx,
-                                                                                 gates, counts, tile_counts,
-                                                                                 tile_psum, status);
+    if constexpr (BAL)
+        router_logits_vec_balance_kernel<K, NV, FULL><<<grid, kThreads, smem, stream>>>(
+            logits, bias, T, Nr, topk_idx, gates, counts, tile_counts, tile_psum, status);
+    else
+        router_logits_vec_kernel<K, NV, FULL><<<grid, kThreads, smem, stream>>>(logits, bias, T, Nr, topk_idx, gates,
+                                                                               counts, tile_counts, status);
     return cudaGetLastError();
 }
 
