@@ -477,14 +477,23 @@ __device__ __forceinline__ void logits_vec_body(const float *__restrict__ logits
                 }
             }
         } else {
+            // key_approx on pairs of columns through the packed two-lane fp32
+            // instructions (each half rounds like the scalar operation)
+            const float2 half = make_float2(0.5f, 0.5f);
 #pragma unroll
             for (int m = 0; m < NV; ++m) {
                 const float4 x = *reinterpret_cast<const float4 *>(xr + 4 * m);
                 const float4 h = *reinterpret_cast<const float4 *>(hbl + 4 * m);
-                kv[m][0] = key_approx(x.x, h.x);
-                kv[m][1] = key_approx(x.y, h.y);
-                kv[m][2] = key_approx(x.z, h.z);
-                kv[m][3] = key_approx(x.w, h.w);
+                const float2 xa = __fmul2_rn(half, make_float2(x.x, x.y));
+                const float2 xb = __fmul2_rn(half, make_float2(x.z, x.w));
+                const float2 ya =
+                    __ffma2_rn(half, make_float2(tanh_approx(xa.x), tanh_approx(xa.y)), make_float2(h.x, h.y));
+                const float2 yb =
+                    __ffma2_rn(half, make_float2(tanh_approx(xb.x), tanh_approx(xb.y)), make_float2(h.z, h.w));
+                kv[m][0] = ya.x;
+                kv[m][1] = ya.y;
+                kv[m][2] = yb.x;
+                kv[m][3] = yb.y;
             }
         }
         // tau': the K-th largest of the maxima of groups of 8 keys (each
@@ -508,15 +517,29 @@ __device__ __forceinline__ void logits_vec_body(const float *__restrict__ logits
                 lo = fminf(a, b);
             };
             if constexpr (G == 2) ce(gm[0], gm[1]);
-            if constexpr (G == 4) {
+            if constexpr (G == 4 && P == 4) {
+                ce(gm[0], gm[1]);
+                ce(gm[2], gm[3]);
+                const float hi = fmaxf(gm[0], gm[2]);
+                gm[1] = fmaxf(fminf(gm[0], gm[2]), fmaxf(gm[1], gm[3]));
+                gm[0] = hi;
+            } else if constexpr (G == 4) {
                 ce(gm[0], gm[1]);
                 ce(gm[2], gm[3]);
                 ce(gm[0], gm[2]);
                 ce(gm[1], gm[3]);
                 ce(gm[1], gm[2]);
             }
+            if constexpr (G == 4 && P == 4) {
+                // K = 3 or 4: the lane's two largest group maxima are enough
+                // (the K-th largest of what the row's lanes keep is still at
+                // most the K-th key); the list's lower two slots stay -inf
+                top.v[0] = gm[0];
+                top.v[1] = gm[1];
+            } else {
 #pragma unroll
-            for (int q = 0; q < G; ++q) top.v[q] = gm[q];
+                for (int q = 0; q < G; ++q) top.v[q] = gm[q];
+            }
         } else {
 #pragma unroll
             for (int q = 0; q < G; ++q) top.push(gm[q]);
