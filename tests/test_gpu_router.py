@@ -226,7 +226,7 @@ def test_logits_mode_all_equal_keys(cuda_device):
 def test_logits_mode_many_tied_candidates(cuda_device, Nr, K, misalign):
     """Rows where 1..90 experts tie at the top key (logits on a 1/8 grid, bias
     on a 1/8 grid for half of the rows): the candidates of a row are scored in
-    one to three rounds of 32 and merged, and equal keys go to the lower
+    one to four rounds of 24 and merged, and equal keys go to the lower
     index."""
     T = 3000
     g = torch.Generator().manual_seed(Nr * 10 + K)
@@ -238,6 +238,35 @@ def test_logits_mode_many_tied_candidates(cuda_device, Nr, K, misalign):
     bias = torch.zeros(Nr)
     bias[torch.randperm(Nr, generator=g)[: Nr // 4]] = -0.125
     idx, gates, counts, tiles = _run_logits(x, bias, K, misalign=misalign)
+    ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
+    assert np.array_equal(idx, ref.idx)
+    assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
+    assert np.array_equal(counts, ref.counts)
+    assert np.array_equal(tiles, ref.tile_counts)
+
+
+@pytest.mark.parametrize("layout", ["spread", "clustered"])
+@pytest.mark.parametrize("Nr,K", [(256, 4), (128, 8), (64, 2), (256, 1)])
+def test_logits_mode_wide_fast_path(cuda_device, Nr, K, layout):
+    """Every row has 5 to 16 experts tied at the top key, spread over the row
+    or packed into runs of consecutive experts (up to 8 in one lane's block
+    of the vector kernel): the loop-free candidate stage then scores two
+    candidates per lane and takes up to 8 from one lane.  Equal keys go to the
+    lower index, bit for bit as the oracle."""
+    T = 4096
+    g = torch.Generator().manual_seed(Nr * 100 + K + (7 if layout == "clustered" else 0))
+    x = torch.round(torch.randn(T, Nr, generator=g) * 8) / 8 - 4.0
+    ties = torch.randint(5, 17, (T,), generator=g)
+    for t in range(T):
+        n = int(ties[t])
+        if layout == "spread":
+            cols = torch.randperm(Nr, generator=g)[:n]
+        else:
+            start = int(torch.randint(0, Nr - n + 1, (1,), generator=g))
+            cols = torch.arange(start, start + n)
+        x[t, cols] = 1.5
+    bias = torch.zeros(Nr)
+    idx, gates, counts, tiles = _run_logits(x, bias, K)
     ref = oracle.router_logits(x.numpy(), bias.numpy(), K, tile_tokens=128)
     assert np.array_equal(idx, ref.idx)
     assert np.array_equal(gates.view(np.uint32), ref.gates.view(np.uint32))
