@@ -572,8 +572,10 @@ def main():
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": profiled_traffic("ties_full"),
                 "kernel": "router_gemm_kernel<4>", "kernel_ms": router_ms,
-                "peak_source": "%s %s bf16 (MEASURED_PEAKS.json); timed loop %.2f s" % (
-                    peaks["source"], "sustained" if long_loop else "burst", total_ms / 1e3),
+                "peak_source": "%s %s bf16 (%s); timed loop %.2f s" % (
+                    peaks["source"], "sustained" if long_loop else "burst",
+                    "MEASURED_PEAKS.json" if peaks["source"] == "measured" else "no MEASURED_PEAKS.json: the pool's earlier figures",
+                    total_ms / 1e3),
                 "frac_of_burst": achieved / peaks["bf16_tflops"],
                 "frac_of_sustained": achieved / sustained if sustained else None,
                 "hbm_view": {"alg_bytes": alg_bytes, "achieved_gbs": alg_bytes / (router_ms / 1e3) / 1e9,
