@@ -244,7 +244,8 @@ __device__ __forceinline__ float tanh_approx(float x) {
     return y;
 }
 
-// The largest of three values; NaN inputs are ignored like fmaxf does.
+// The largest of three values in one three-input max instruction (the keys
+// it compares are finite or -inf; inputs are assumed finite).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float y;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
